@@ -1,0 +1,202 @@
+// CPU oracle for the DSA forward path: plain, slow, fp64.
+//
+// TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the bench's
+// CPU-baseline leg may load this library. The CUDA library never links,
+// includes or calls it, and it shares no code with the CUDA library.
+//
+// What it computes (page "DeepseekV3.2 拆解", section "核心组件"):
+//   * lightning indexer score, equation I_{t,s}:
+//       I[t,s] = sum_j w[t,j] * ReLU(q[t,j] . k[s]),  j = 1..H^I,
+//     with q and k the dequantised FP8 vectors (code value * per-row scale);
+//   * fine-grained token selection, equation u_t = Attn(h_t, {c_s | I_{t,s}
+//     in Top-k(I_{t,:})}): the k keys with the largest score, ties broken by
+//     the lower key index, fewer than k valid keys -> all of them, pad -1;
+//   * the attention over the selected latent rows c_s (MQA: every query head
+//     reads the same row; K = all qk_dim dims, V = the first v_dim dims; the
+//     latent width 576 = 512 + 64 follows the MLA section 1.1 of page
+//     "DeepSeek architecture"), exact softmax in fp64.
+// Everything is the definition written out: no blocking, no fusion, no
+// reordering of the sums beyond the natural loop order.
+//
+// Parity pins live in tests/test_oracle.py (closed forms, library special
+// cases, brute force, invariants); the pages print no worked example.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <thread>
+#include <vector>
+
+namespace {
+
+// OCP 8-bit floating point, E4M3 ("fn" flavour): 1 sign bit, 4 exponent bits
+// with bias 7, 3 mantissa bits; exponent field 0 is subnormal; S.1111.111 is
+// NaN; there is no infinity.
+double e4m3_value(uint8_t code) {
+  const int sign = (code >> 7) & 1;
+  const int e = (code >> 3) & 0xF;
+  const int m = code & 0x7;
+  double mag;
+  if (e == 0xF && m == 0x7) return std::numeric_limits<double>::quiet_NaN();
+  if (e == 0) {
+    mag = std::ldexp(static_cast<double>(m) / 8.0, 1 - 7);
+  } else {
+    mag = std::ldexp(1.0 + static_cast<double>(m) / 8.0, e - 7);
+  }
+  return sign ? -mag : mag;
+}
+
+// bfloat16 is the upper half of an IEEE binary32.
+double bf16_value(uint16_t bits) {
+  uint32_t u = static_cast<uint32_t>(bits) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof(f));
+  return static_cast<double>(f);
+}
+
+template <class F>
+void parallel_rows(int n_rows, int n_threads, F&& body) {
+  if (n_threads <= 0) n_threads = static_cast<int>(std::thread::hardware_concurrency());
+  if (n_threads <= 0) n_threads = 1;
+  n_threads = std::min(n_threads, std::max(n_rows, 1));
+  if (n_threads == 1) {
+    for (int r = 0; r < n_rows; ++r) body(r);
+    return;
+  }
+  std::vector<std::thread> pool;
+  for (int th = 0; th < n_threads; ++th) {
+    pool.emplace_back([&, th]() {
+      for (int r = th; r < n_rows; r += n_threads) body(r);
+    });
+  }
+  for (auto& t : pool) t.join();
+}
+
+}  // namespace
+
+extern "C" {
+
+int oracle_hardware_threads() {
+  return static_cast<int>(std::thread::hardware_concurrency());
+}
+
+double oracle_e4m3_value(uint8_t code) { return e4m3_value(code); }
+
+// Indexer scores for n_rows query rows of ONE sequence.
+//   q8   [n_rows, HI, DI] e4m3 codes,  qs [n_rows, HI] scale per (row, head)
+//   w    [n_rows, HI]
+//   k8   [S, DI] e4m3 codes,           ks [S] scale per key
+//   pos  [n_rows] absolute query position of each row
+//   kv_len: keys with index >= kv_len are invalid
+//   out  [n_rows, S]: I[t,s] for valid s (s <= pos and s < kv_len), -inf else
+void oracle_indexer_scores(int n_rows, int S, int HI, int DI,
+                           const uint8_t* q8, const float* qs, const float* w,
+                           const uint8_t* k8, const float* ks,
+                           const int32_t* pos, int kv_len,
+                           double* out, int n_threads) {
+  const double neg_inf = -std::numeric_limits<double>::infinity();
+  parallel_rows(n_rows, n_threads, [&](int r) {
+    std::vector<double> qhat(static_cast<size_t>(HI) * DI);
+    for (int j = 0; j < HI; ++j)
+      for (int d = 0; d < DI; ++d)
+        qhat[static_cast<size_t>(j) * DI + d] =
+            e4m3_value(q8[(static_cast<size_t>(r) * HI + j) * DI + d]) *
+            static_cast<double>(qs[static_cast<size_t>(r) * HI + j]);
+    std::vector<double> khat(DI);
+    double* row_out = out + static_cast<size_t>(r) * S;
+    for (int s = 0; s < S; ++s) {
+      if (s > pos[r] || s >= kv_len) {
+        row_out[s] = neg_inf;
+        continue;
+      }
+      for (int d = 0; d < DI; ++d)
+        khat[d] = e4m3_value(k8[static_cast<size_t>(s) * DI + d]) *
+                  static_cast<double>(ks[s]);
+      double score = 0.0;
+      for (int j = 0; j < HI; ++j) {
+        double dot = 0.0;
+        for (int d = 0; d < DI; ++d) dot += qhat[static_cast<size_t>(j) * DI + d] * khat[d];
+        const double relu = dot > 0.0 ? dot : 0.0;
+        score += static_cast<double>(w[static_cast<size_t>(r) * HI + j]) * relu;
+      }
+      row_out[s] = score;
+    }
+  });
+}
+
+// Top-k selection per row: sort the valid keys (finite score) by
+// (score descending, index ascending) and keep the first min(k, #valid);
+// remaining slots are -1.
+//   scores [n_rows, S], out [n_rows, k]
+void oracle_topk(int n_rows, int S, int k, const double* scores, int32_t* out,
+                 int n_threads) {
+  parallel_rows(n_rows, n_threads, [&](int r) {
+    const double* row = scores + static_cast<size_t>(r) * S;
+    std::vector<int32_t> cand;
+    cand.reserve(S);
+    for (int s = 0; s < S; ++s)
+      if (std::isfinite(row[s])) cand.push_back(s);
+    std::sort(cand.begin(), cand.end(), [row](int32_t a, int32_t b) {
+      if (row[a] != row[b]) return row[a] > row[b];
+      return a < b;
+    });
+    int32_t* o = out + static_cast<size_t>(r) * k;
+    for (int i = 0; i < k; ++i)
+      o[i] = i < static_cast<int>(cand.size()) ? cand[i] : -1;
+  });
+}
+
+// Attention of n_rows query rows of ONE sequence over their selected latent
+// rows.
+//   q    [n_rows, H, Dqk] bf16 bits
+//   kv   [S, Dqk] bf16 bits; K = kv[s, 0:Dqk], V = kv[s, 0:Dv]
+//   idx  [n_rows, k] selected key indices, -1 = empty slot
+//   o    [n_rows, H, Dv]; lse [n_rows, H] (natural log)
+// A row with no selected key gets o = 0 and lse = -inf.
+void oracle_sparse_attn(int n_rows, int S, int H, int Dqk, int Dv, int k,
+                        double scale, const uint16_t* q, const uint16_t* kv,
+                        const int32_t* idx, double* o, double* lse,
+                        int n_threads) {
+  parallel_rows(n_rows, n_threads, [&](int r) {
+    const int32_t* sel = idx + static_cast<size_t>(r) * k;
+    std::vector<int32_t> keys;
+    for (int i = 0; i < k; ++i)
+      if (sel[i] >= 0 && sel[i] < S) keys.push_back(sel[i]);
+    const int n = static_cast<int>(keys.size());
+    std::vector<double> z(n), qh(Dqk);
+    for (int h = 0; h < H; ++h) {
+      double* oh = o + (static_cast<size_t>(r) * H + h) * Dv;
+      for (int d = 0; d < Dqk; ++d)
+        qh[d] = bf16_value(q[(static_cast<size_t>(r) * H + h) * Dqk + d]);
+      if (n == 0) {
+        for (int d = 0; d < Dv; ++d) oh[d] = 0.0;
+        lse[static_cast<size_t>(r) * H + h] = -std::numeric_limits<double>::infinity();
+        continue;
+      }
+      double m = -std::numeric_limits<double>::infinity();
+      for (int i = 0; i < n; ++i) {
+        const uint16_t* c = kv + static_cast<size_t>(keys[i]) * Dqk;
+        double dot = 0.0;
+        for (int d = 0; d < Dqk; ++d) dot += qh[d] * bf16_value(c[d]);
+        z[i] = scale * dot;
+        m = std::max(m, z[i]);
+      }
+      double l = 0.0;
+      for (int i = 0; i < n; ++i) {
+        z[i] = std::exp(z[i] - m);
+        l += z[i];
+      }
+      for (int d = 0; d < Dv; ++d) oh[d] = 0.0;
+      for (int i = 0; i < n; ++i) {
+        const uint16_t* c = kv + static_cast<size_t>(keys[i]) * Dqk;
+        const double p = z[i] / l;
+        for (int d = 0; d < Dv; ++d) oh[d] += p * bf16_value(c[d]);
+      }
+      lse[static_cast<size_t>(r) * H + h] = m + std::log(l);
+    }
+  });
+}
+
+}  // extern "C"

@@ -1,0 +1,291 @@
+"""Pins for the fp64 CPU oracle, independent of the oracle's own code.
+
+Each test checks the oracle against something fixed outside it: the OCP E4M3
+definition and torch's float8 cast, closed-form identities of ReLU, library
+routines (torch matmul / scaled_dot_product_attention / logsumexp) on special
+cases, brute-force rank counting, and invariants the method implies (page
+"DeepseekV3.2 拆解", section "核心组件": the indexer equation I_{t,s} and the
+selection equation u_t = Attn(h_t, {c_s | I_{t,s} in Top-k(I_{t,:})})).
+A plausible slip in the oracle (dropped term, wrong sign, wrong index,
+transposed operand, wrong tie rule) fails at least one test here.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from sparse_attention_long_fp8_b200 import inputs as dsa_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _decode_fp8_torch(codes_u8):
+    return codes_u8.view(torch.float8_e4m3fn).to(torch.float64)
+
+
+def _bf16_to_f64(x):
+    return x.to(torch.float64)
+
+
+def _small_indexer(seed, n, S, HI, DI, w_pos=False):
+    g = torch.Generator().manual_seed(seed)
+    q8, qs = dsa_inputs.quantize_e4m3_rows(torch.randn(n, HI, DI, generator=g))
+    k8, ks = dsa_inputs.quantize_e4m3_rows(torch.randn(S, DI, generator=g))
+    w = torch.randn(n, HI, generator=g)
+    if w_pos:
+        w = w.abs()
+    return q8, qs, w, k8, ks
+
+
+# ---------------------------------------------------------------- e4m3 decode
+
+def test_e4m3_golden_points(oracle_lib):
+    path = os.path.join(GOLDEN, "e4m3_ocp_points.txt")
+    n = 0
+    for line in open(path, encoding="utf-8"):
+        if not line.strip() or line.startswith("#"):
+            continue
+        code, val = line.split()
+        got = oracle_lib.e4m3_value(int(code, 16))
+        if val == "nan":
+            assert math.isnan(got)
+        else:
+            assert got == float(val) and math.copysign(1, got) == math.copysign(1, float(val))
+        n += 1
+    assert n >= 10
+
+
+def test_e4m3_exhaustive_vs_torch(oracle_lib):
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for c in range(256):
+        got = oracle_lib.e4m3_value(c)
+        if math.isnan(ref[c]):
+            assert math.isnan(got), c
+        else:
+            assert got == ref[c], (c, got, ref[c])
+
+
+# ---------------------------------------------------------------- indexer
+
+def test_indexer_single_head_is_relu_matmul(oracle_lib):
+    """H^I = 1, w = 1, unit scales: I[t,s] = ReLU(q_t . k_s), a plain matmul."""
+    n, S, DI = 9, 13, 32
+    q8, _, _, k8, _ = _small_indexer(1, n, S, 1, DI)
+    qs = torch.ones(n, 1); ks = torch.ones(S); w = torch.ones(n, 1)
+    pos = np.arange(n, dtype=np.int32) + 3
+    got = oracle_lib.indexer_scores(q8, qs, w, k8, ks, pos, kv_len=S)
+    dots = _decode_fp8_torch(q8[:, 0, :]) @ _decode_fp8_torch(k8).T
+    ref = torch.relu(dots).numpy()
+    for t in range(n):
+        for s in range(S):
+            if s <= pos[t]:
+                assert got[t, s] == pytest.approx(ref[t, s], rel=1e-12, abs=1e-9)
+            else:
+                assert got[t, s] == -np.inf
+
+
+def _flip_sign(codes):
+    return codes ^ torch.tensor(0x80, dtype=torch.uint8)
+
+
+@pytest.mark.parametrize("HI,DI", [(4, 32), (64, 128)])
+def test_indexer_relu_identities(oracle_lib, HI, DI):
+    """ReLU(x) - ReLU(-x) = x and ReLU(x) + ReLU(-x) = |x| give two closed
+    forms: I(q) - I(-q) = sum_j w_j x_j and I(q) + I(-q) = sum_j w_j |x_j|,
+    with x_j = (qs_j q_j) . (ks_s k_s) computed by a library matmul."""
+    n, S = 6, 20
+    q8, qs, w, k8, ks = _small_indexer(2, n, S, HI, DI)
+    pos = np.full(n, S - 1, dtype=np.int32)
+    i_pos = oracle_lib.indexer_scores(q8, qs, w, k8, ks, pos, S)
+    i_neg = oracle_lib.indexer_scores(_flip_sign(q8), qs, w, k8, ks, pos, S)
+    qhat = _decode_fp8_torch(q8) * qs.double()[..., None]          # [n, HI, DI]
+    khat = _decode_fp8_torch(k8) * ks.double()[:, None]            # [S, DI]
+    x = torch.einsum("njd,sd->njs", qhat, khat)                    # [n, HI, S]
+    lin = (w.double()[..., None] * x).sum(1).numpy()
+    absum = (w.double()[..., None] * x.abs()).sum(1).numpy()
+    scale = np.abs(absum).max()
+    np.testing.assert_allclose(i_pos - i_neg, lin, rtol=0, atol=1e-12 * scale)
+    np.testing.assert_allclose(i_pos + i_neg, absum, rtol=0, atol=1e-12 * scale)
+
+
+def test_indexer_head_terms_nonnegative(oracle_lib):
+    """Every head term w_j * ReLU(.) has the sign of w_j: w >= 0 gives I >= 0,
+    w <= 0 gives I <= 0, and a single head with w = 1 is >= 0."""
+    n, S, HI, DI = 5, 16, 4, 32
+    q8, qs, w, k8, ks = _small_indexer(3, n, S, HI, DI, w_pos=True)
+    pos = np.full(n, S - 1, dtype=np.int32)
+    assert (oracle_lib.indexer_scores(q8, qs, w, k8, ks, pos, S) >= 0).all()
+    assert (oracle_lib.indexer_scores(q8, qs, -w, k8, ks, pos, S) <= 0).all()
+
+
+def test_indexer_head_permutation_invariance(oracle_lib):
+    n, S, HI, DI = 4, 24, 64, 128
+    q8, qs, w, k8, ks = _small_indexer(4, n, S, HI, DI)
+    pos = np.arange(n, dtype=np.int32) * 5
+    perm = torch.randperm(HI, generator=torch.Generator().manual_seed(9))
+    a = oracle_lib.indexer_scores(q8, qs, w, k8, ks, pos, S)
+    b = oracle_lib.indexer_scores(q8[:, perm], qs[:, perm], w[:, perm], k8, ks, pos, S)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
+
+
+def test_indexer_linear_in_w_and_homogeneous_in_scales(oracle_lib):
+    n, S, HI, DI = 4, 18, 4, 32
+    q8, qs, _, k8, ks = _small_indexer(5, n, S, HI, DI)
+    # dyadic weights keep w + w2 exact in fp32
+    gw = torch.Generator().manual_seed(6)
+    w = torch.randint(-8, 9, (n, HI), generator=gw).float() / 8
+    w2 = torch.randint(-8, 9, (n, HI), generator=gw).float() / 8
+    pos = np.full(n, S - 1, dtype=np.int32)
+    f = lambda **kw: oracle_lib.indexer_scores(kw.get("q8", q8), kw.get("qs", qs),
+                                               kw.get("w", w), k8, kw.get("ks", ks), pos, S)
+    base = f()
+    tol = 1e-12 * np.abs(base).max()
+    np.testing.assert_allclose(f(w=w + w2), base + f(w=w2), rtol=0, atol=10 * tol)
+    np.testing.assert_allclose(f(qs=qs * 4.0), 4.0 * base, rtol=0, atol=10 * tol)
+    np.testing.assert_allclose(f(ks=ks * 0.25), 0.25 * base, rtol=0, atol=10 * tol)
+    # scaling one head's q-scale scales only that head's term
+    qs1 = qs.clone(); qs1[:, 2] *= 2.0
+    w_only2 = torch.zeros_like(w); w_only2[:, 2] = w[:, 2]
+    np.testing.assert_allclose(f(qs=qs1) - base, f(w=w_only2), rtol=0, atol=10 * tol)
+
+
+def test_indexer_mask_causal_and_kv_len(oracle_lib):
+    n, S, HI, DI = 6, 30, 4, 32
+    q8, qs, w, k8, ks = _small_indexer(7, n, S, HI, DI)
+    pos = np.array([0, 3, 10, 25, 29, 40], dtype=np.int32)
+    kv_len = 27
+    sc = oracle_lib.indexer_scores(q8, qs, w, k8, ks, pos, kv_len)
+    for t in range(n):
+        for s in range(S):
+            assert np.isfinite(sc[t, s]) == (s <= pos[t] and s < kv_len)
+
+
+# ---------------------------------------------------------------- top-k
+
+def _rank_count_topk(row, k):
+    """s is selected iff fewer than k valid keys beat it, where s' beats s when
+    its score is higher, or equal with a lower index."""
+    valid = [s for s in range(len(row)) if np.isfinite(row[s])]
+    sel = set()
+    for s in valid:
+        beats = sum(1 for s2 in valid if row[s2] > row[s] or (row[s2] == row[s] and s2 < s))
+        if beats < k:
+            sel.add(s)
+    return sel
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_topk_brute_force_rank_count(oracle_lib, seed):
+    rng = np.random.default_rng(seed)
+    L = int(rng.integers(1, 13))
+    k = int(rng.integers(1, 15))
+    # coarse values force ties; some -inf entries are invalid keys
+    scores = rng.integers(-3, 4, size=(4, L)).astype(np.float64)
+    scores[rng.random((4, L)) < 0.2] = -np.inf
+    got = oracle_lib.topk(scores, k)
+    for r in range(4):
+        want = _rank_count_topk(scores[r], k)
+        sel = [int(i) for i in got[r] if i >= 0]
+        assert len(sel) == len(set(sel)) == len(want)
+        assert set(sel) == want
+        # the -1 pads come last
+        assert all(i == -1 for i in got[r][len(sel):])
+
+
+def test_topk_all_ties_take_lowest_indices(oracle_lib):
+    scores = np.zeros((2, 50))
+    got = oracle_lib.topk(scores, 7)
+    assert sorted(got[0].tolist()) == list(range(7))
+
+
+# ---------------------------------------------------------------- attention
+
+def _attn_case(seed, n, S, H, Dqk):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(n, H, Dqk, generator=g).to(torch.bfloat16)
+    kv = torch.randn(S, Dqk, generator=g).to(torch.bfloat16)
+    return q, kv
+
+
+@pytest.mark.parametrize("Dqk,Dv", [(64, 64), (64, 48)])
+def test_attn_full_set_equals_dense_causal_sdpa(oracle_lib, Dqk, Dv):
+    """k >= t+1: the selection keeps every causal key, so the result is dense
+    causal attention (torch SDPA in float64 as the textbook reference)."""
+    T, H = 12, 8
+    q, kv = _attn_case(11, T, T, H, Dqk)
+    scale = 0.125
+    idx = np.full((T, T + 3), -1, dtype=np.int32)
+    rng = np.random.default_rng(0)
+    for t in range(T):
+        idx[t, : t + 1] = rng.permutation(t + 1)
+    o, lse = oracle_lib.sparse_attn(q, kv, idx, scale, Dv)
+    qd = _bf16_to_f64(q).permute(1, 0, 2)[None]                       # [1, H, T, D]
+    kd = _bf16_to_f64(kv)[None, None].expand(1, H, T, Dqk)
+    vd = _bf16_to_f64(kv)[:, :Dv][None, None].expand(1, H, T, Dv)
+    ref = torch.nn.functional.scaled_dot_product_attention(qd, kd, vd, is_causal=True, scale=scale)
+    np.testing.assert_allclose(o, ref[0].permute(1, 0, 2).numpy(), rtol=0, atol=1e-12)
+    z = (qd @ kd.transpose(-1, -2)) * scale
+    z = z.masked_fill(torch.triu(torch.ones(T, T, dtype=torch.bool), 1), -math.inf)
+    np.testing.assert_allclose(lse, torch.logsumexp(z, -1)[0].T.numpy(), rtol=0, atol=1e-12)
+
+
+def test_attn_zero_scale_is_mean_of_rows(oracle_lib):
+    q, kv = _attn_case(12, 3, 40, 4, 64)
+    idx = np.array([[5, 1, 9, -1], [0, -1, -1, -1], [39, 38, 2, 17]], dtype=np.int32)
+    o, lse = oracle_lib.sparse_attn(q, kv, idx, 0.0, 64)
+    kvd = _bf16_to_f64(kv).numpy()
+    for r in range(3):
+        rows = [i for i in idx[r] if i >= 0]
+        for h in range(4):
+            np.testing.assert_allclose(o[r, h], kvd[rows].mean(0), rtol=0, atol=1e-12)
+            assert lse[r, h] == pytest.approx(math.log(len(rows)), abs=1e-12)
+
+
+def test_attn_single_key_and_empty_set(oracle_lib):
+    q, kv = _attn_case(13, 2, 10, 3, 64)
+    idx = np.array([[4, -1], [-1, -1]], dtype=np.int32)
+    o, lse = oracle_lib.sparse_attn(q, kv, idx, 0.3, 32)
+    kvd = _bf16_to_f64(kv).numpy(); qd = _bf16_to_f64(q).numpy()
+    for h in range(3):
+        np.testing.assert_allclose(o[0, h], kvd[4, :32], rtol=0, atol=0)
+        assert lse[0, h] == pytest.approx(0.3 * float(qd[0, h] @ kvd[4]), rel=1e-12)
+        assert (o[1, h] == 0).all() and lse[1, h] == -np.inf
+
+
+def test_attn_slot_order_irrelevant(oracle_lib):
+    q, kv = _attn_case(14, 2, 64, 8, 64)
+    idx = np.stack([np.arange(0, 64, 3)[:16], np.arange(1, 64, 4)[:16]]).astype(np.int32)
+    o1, l1 = oracle_lib.sparse_attn(q, kv, idx, 0.125, 64)
+    o2, l2 = oracle_lib.sparse_attn(q, kv, idx[:, ::-1].copy(), 0.125, 64)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------- full path
+
+def test_forward_tiny_invariants(oracle_lib):
+    """Tiny config: selections are causal, sized min(k, t+1), and the first k
+    rows (where k >= t+1) equal dense causal attention."""
+    cfg = dsa_inputs.CONFIGS["tiny"]
+    inp = dsa_inputs.make_inputs(cfg, seed=0)
+    rows = np.array([0, 1, 2, 30, 62, 63, 64, 65, 130, 255])
+    res = oracle_lib.forward(inp, cfg, rows=rows)
+    for r, t in enumerate(rows):
+        sel = res["indices"][r]
+        valid = sel[sel >= 0]
+        assert len(valid) == min(cfg.topk, t + 1)
+        assert (valid <= t).all() and len(set(valid.tolist())) == len(valid)
+    dense_rows = rows[rows + 1 <= cfg.topk]
+    q = inp["q"][0]; kv = inp["kv"][0]
+    H, D = cfg.heads, cfg.qk_dim
+    for r, t in enumerate(rows):
+        if t + 1 > cfg.topk:
+            continue
+        qd = _bf16_to_f64(q[t])                                      # [H, D]
+        kd = _bf16_to_f64(kv[: t + 1])                               # [t+1, D]
+        p = torch.softmax(qd @ kd.T * cfg.softmax_scale, -1)
+        np.testing.assert_allclose(res["o"][r], (p @ kd[:, : cfg.v_dim]).numpy(), rtol=0, atol=1e-12)
+    assert len(dense_rows) > 0
