@@ -1,0 +1,171 @@
+/*
+ * dsa.h - C ABI of the DeepSeek Sparse Attention (DSA) forward path on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method (page "DeepseekV3.2 拆解", section "核心组件"):
+ *   lightning indexer   I[t,s] = sum_{j=1..H^I} w[t,j] * ReLU(q[t,j] . k[s])
+ *                       over FP8 indexer queries/keys ("闪电索引器", eq. I_{t,s});
+ *   token selection     S_t = Top-k(I[t,:]), k = 2048 in the deployed model
+ *                       ("细粒度 Token 选择机制" and the complexity table row
+ *                       "DSA 核心注意力");
+ *   core attention      u_t = Attn(h_t, {c_s : s in S_t}) over the MLA latent
+ *                       rows c_s (eq. u_t); the latent is 576 wide = 512
+ *                       value dims + 64 decoupled-RoPE dims (page "DeepSeek
+ *                       architecture", section 1.1, "4.5 d_h l" per token).
+ *
+ * Conventions shared by every call
+ *   - Every pointer argument is a DEVICE pointer, allocated and owned by the
+ *     caller. The library allocates no device memory and keeps no pointer
+ *     after a call returns.
+ *   - Every call is asynchronous on the caller's CUDA stream (`stream`, a
+ *     cudaStream_t passed as void*; NULL = legacy default stream). No call
+ *     synchronises except dsa_check().
+ *   - Argument errors are detected on the host BEFORE any launch and reported
+ *     by the return value; dsa_last_error() gives a one-line reason.
+ *   - Device-side failures (a bounded wait that ran out) set a per-device
+ *     error word that dsa_check() reads and clears. Kernels never trap.
+ *   - Scales (q_scale, k_scale) must be finite and > 0 (amax/448, or 1 for an
+ *     all-zero row); the kernels rely on ReLU(a*x) = a*ReLU(x) for a > 0.
+ *   - Validity: key s is visible to query row i of sequence b iff
+ *       s <= q_pos0[b] + i  and  s < kv_len[b].
+ *     q_pos0 / kv_len are device int32 [batch] arrays, or NULL for
+ *     q_pos0 = 0 (prefill from position 0) and kv_len = n_kv.
+ *     Decode: n_q = 1 and q_pos0[b] = kv_len[b] - 1.
+ *   - Supported shapes (others return DSA_ERR_UNSUPPORTED):
+ *       (idx_heads, idx_dim) in {(64, 128), (4, 32)};
+ *       (heads, qk_dim, v_dim) in {(128, 576, 512), (8, 64, 64)};
+ *       1 <= topk; n_q, n_kv >= 1; batch >= 1.
+ */
+#ifndef DSA_B200_DSA_H_
+#define DSA_B200_DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, row range, ...      */
+  DSA_ERR_UNSUPPORTED = 2,  /* shape outside the compiled tile set         */
+  DSA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required  */
+  DSA_ERR_CUDA = 4,         /* a CUDA runtime call failed                  */
+  DSA_ERR_TIMEOUT = 5,      /* a device-side bounded wait ran out          */
+  DSA_ERR_NO_DEVICE = 6     /* no sm_100 device is current                 */
+} dsa_status;
+
+typedef enum { DSA_OUT_F32 = 0, DSA_OUT_BF16 = 1 } dsa_out_dtype;
+
+typedef enum {
+  DSA_OP_INDEXER = 0,
+  DSA_OP_TOPK = 1,
+  DSA_OP_SPARSE_ATTN = 2,
+  DSA_OP_FORWARD = 3
+} dsa_op;
+
+typedef struct {
+  int32_t batch;          /* B                                              */
+  int32_t n_q;            /* query rows per sequence (T)                    */
+  int32_t n_kv;           /* key / latent rows per sequence (S)             */
+  int32_t idx_heads;      /* H^I, indexer heads                             */
+  int32_t idx_dim;        /* d^I, indexer head dim (bytes per fp8 row)      */
+  int32_t topk;           /* k                                              */
+  int32_t heads;          /* H, attention query heads (share one latent)    */
+  int32_t qk_dim;         /* D_qk, dims of q and of the latent row          */
+  int32_t v_dim;          /* D_v, value dims = the first v_dim latent dims  */
+  float softmax_scale;    /* logits = softmax_scale * q . c                 */
+} dsa_shape;
+
+/*
+ * Indexer scores (page "DeepseekV3.2 拆解", eq. I_{t,s}), materialised.
+ *   q_fp8   [B, n_q, H^I, d^I] e4m3fn codes     q_scale [B, n_q, H^I] fp32
+ *   w       [B, n_q, H^I] fp32 head weights
+ *   k_fp8   [B, n_kv, d^I] e4m3fn codes         k_scale [B, n_kv] fp32
+ *   rows [row_begin, row_end) of every sequence are scored:
+ *   scores  [B, row_end-row_begin, n_kv] fp32; invisible keys get -inf.
+ *   I[t,s] = k_scale[s] * sum_j (w[t,j] q_scale[t,j]) ReLU(q8[t,j] . k8[s]),
+ *   the dot products exact-product / fp32-accumulated on the tensor cores.
+ */
+dsa_status dsa_indexer_scores(const dsa_shape* shape, const uint8_t* q_fp8,
+                              const float* q_scale, const float* w,
+                              const uint8_t* k_fp8, const float* k_scale,
+                              const int32_t* q_pos0, const int32_t* kv_len,
+                              int32_t row_begin, int32_t row_end,
+                              float* scores, void* stream);
+
+/*
+ * Top-k selection per score row (page "DeepseekV3.2 拆解", eq. u_t: keep the
+ * k keys with the largest I[t,s]).
+ *   scores  [B, row_end-row_begin, n_kv] fp32 (as written by
+ *           dsa_indexer_scores for the same rows); only the visible keys of
+ *           each row are read.
+ *   indices [B, row_end-row_begin, topk] int32. A row with m visible keys
+ *           gets min(m, topk) distinct key indices, then -1 padding. Among
+ *           equal scores the lower key index wins. The order of the
+ *           selected indices within a row is unspecified.
+ *   No workspace is needed (ws may be NULL, ws_bytes 0).
+ */
+dsa_status dsa_topk(const dsa_shape* shape, const float* scores,
+                    int32_t row_begin, int32_t row_end,
+                    const int32_t* q_pos0, const int32_t* kv_len,
+                    int32_t* indices, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Sparse MQA attention over the selected latent rows (eq. u_t).
+ *   q       [B, n_q, H, D_qk] bf16
+ *   kv      [B, n_kv, D_qk] bf16 latent rows; K = kv[s, :D_qk],
+ *           V = kv[s, :D_v], shared by all H heads
+ *   indices [B, n_q, topk] int32 key indices into kv of the same sequence,
+ *           -1 = empty slot (skipped). Indices outside [0, n_kv) are treated
+ *           as empty.
+ *   out     [B, n_q, H, D_v] fp32 or bf16 (out_dtype)
+ *   lse     [B, n_q, H] fp32 natural-log sum of exp of the logits, or NULL.
+ *   p = softmax(softmax_scale * q . K) over the row's slots, out = p V.
+ *   A row with no valid slot gets out = 0 and lse = -inf.
+ *   Workspace: dsa_workspace_size(shape, DSA_OP_SPARSE_ATTN) bytes (split-K
+ *   partials for short query counts), 256-byte aligned.
+ */
+dsa_status dsa_sparse_attn(const dsa_shape* shape, const uint16_t* q,
+                           const uint16_t* kv, const int32_t* indices,
+                           void* out, int32_t out_dtype, float* lse,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The whole path for all n_q rows: indexer -> top-k -> sparse attention.
+ *   Indexer inputs as dsa_indexer_scores, attention inputs as
+ *   dsa_sparse_attn. indices_out [B, n_q, topk] receives the selection
+ *   (required). Workspace: dsa_workspace_size(shape, DSA_OP_FORWARD).
+ */
+dsa_status dsa_forward(const dsa_shape* shape, const uint8_t* q_fp8,
+                       const float* q_scale, const float* w,
+                       const uint8_t* k_fp8, const float* k_scale,
+                       const int32_t* q_pos0, const int32_t* kv_len,
+                       const uint16_t* q, const uint16_t* kv,
+                       int32_t* indices_out, void* out, int32_t out_dtype,
+                       float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes an op needs for this shape (0 if none). Returns status. */
+dsa_status dsa_workspace_size(const dsa_shape* shape, int32_t op,
+                              size_t* bytes);
+
+/* Synchronises `stream`, then returns DSA_ERR_CUDA for a pending CUDA error,
+ * DSA_ERR_TIMEOUT if a kernel's bounded wait ran out since the last check
+ * (the error word is cleared), else DSA_OK. */
+dsa_status dsa_check(void* stream);
+
+/* Static description of a status code. */
+const char* dsa_status_string(dsa_status status);
+
+/* Reason for the last non-OK status returned on this host thread. */
+const char* dsa_last_error(void);
+
+/* Library version, e.g. "0.1.0". */
+const char* dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_B200_DSA_H_ */

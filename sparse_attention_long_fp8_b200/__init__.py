@@ -1,0 +1,211 @@
+"""DeepSeek Sparse Attention forward path on B200 (sm_100a).
+
+Thin ctypes binding over the C ABI in ``include/dsa.h`` (libdsa.so). Every
+step of the path runs in the library's CUDA kernels; this module only checks
+tensor dtypes/devices, passes raw pointers and turns status codes into
+exceptions. There is no CPU fallback: if the library is missing, importing a
+call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .inputs import CONFIGS, DsaConfig, custom_config, make_inputs  # noqa: F401
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdsa.so")
+
+DSA_OK = 0
+DSA_ERR_INVALID_ARG = 1
+DSA_ERR_UNSUPPORTED = 2
+DSA_ERR_WORKSPACE = 3
+DSA_ERR_CUDA = 4
+DSA_ERR_TIMEOUT = 5
+DSA_ERR_NO_DEVICE = 6
+
+DSA_OUT_F32 = 0
+DSA_OUT_BF16 = 1
+
+DSA_OP_INDEXER = 0
+DSA_OP_TOPK = 1
+DSA_OP_SPARSE_ATTN = 2
+DSA_OP_FORWARD = 3
+
+
+class DsaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"[{status}] {message}")
+        self.status = status
+
+
+class DsaShape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q", ctypes.c_int32), ("n_kv", ctypes.c_int32),
+                ("idx_heads", ctypes.c_int32), ("idx_dim", ctypes.c_int32),
+                ("topk", ctypes.c_int32), ("heads", ctypes.c_int32),
+                ("qk_dim", ctypes.c_int32), ("v_dim", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float)]
+
+
+_lib = None
+
+
+def load_library(path: str | None = None):
+    """Load libdsa.so (built by ``python -m sparse_attention_long_fp8_b200.build``)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m sparse_attention_long_fp8_b200.build`")
+    try:  # share torch's CUDA runtime when torch is present
+        import torch  # noqa: F401
+    except ImportError:
+        pass
+    lib = ctypes.CDLL(path)
+    P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    SP = ctypes.POINTER(DsaShape)
+    lib.dsa_indexer_scores.argtypes = [SP, P, P, P, P, P, P, P, I32, I32, P, P]
+    lib.dsa_topk.argtypes = [SP, P, I32, I32, P, P, P, P, SZ, P]
+    lib.dsa_sparse_attn.argtypes = [SP, P, P, P, P, I32, P, P, SZ, P]
+    lib.dsa_forward.argtypes = [SP, P, P, P, P, P, P, P, P, P, P, P, I32, P, P, SZ, P]
+    lib.dsa_workspace_size.argtypes = [SP, I32, ctypes.POINTER(SZ)]
+    lib.dsa_check.argtypes = [P]
+    lib.dsa_status_string.argtypes = [ctypes.c_int]
+    lib.dsa_status_string.restype = ctypes.c_char_p
+    lib.dsa_last_error.restype = ctypes.c_char_p
+    lib.dsa_version.restype = ctypes.c_char_p
+    for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
+               "dsa_workspace_size", "dsa_check"):
+        getattr(lib, fn).restype = ctypes.c_int
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def _raise(status: int):
+    if status != DSA_OK:
+        lib = load_library()
+        msg = lib.dsa_last_error().decode() or lib.dsa_status_string(status).decode()
+        raise DsaError(status, msg)
+
+
+def shape_of(cfg: DsaConfig) -> DsaShape:
+    return DsaShape(cfg.batch, cfg.n_q, cfg.n_kv, cfg.idx_heads, cfg.idx_dim, cfg.topk,
+                    cfg.heads, cfg.qk_dim, cfg.v_dim, cfg.softmax_scale)
+
+
+def _ptr(t, dtype=None, what="tensor"):
+    """Raw device pointer of a contiguous CUDA tensor (or None -> NULL)."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if dtype is not None and t.dtype not in dtype:
+        raise ValueError(f"{what} has dtype {t.dtype}, expected one of {dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _dt():
+    import torch
+    return {
+        "u8": (torch.uint8, torch.float8_e4m3fn), "f32": (torch.float32,),
+        "i32": (torch.int32,), "bf16": (torch.bfloat16, torch.int16),
+    }
+
+
+def workspace_size(shape: DsaShape, op: int) -> int:
+    n = ctypes.c_size_t(0)
+    _raise(load_library().dsa_workspace_size(ctypes.byref(shape), op, ctypes.byref(n)))
+    return n.value
+
+
+def dsa_indexer_scores(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+                       row_begin, row_end, scores, stream=None):
+    d = _dt()
+    _raise(load_library().dsa_indexer_scores(
+        ctypes.byref(shape), _ptr(q_fp8, d["u8"], "q_fp8"), _ptr(q_scale, d["f32"], "q_scale"),
+        _ptr(w, d["f32"], "w"), _ptr(k_fp8, d["u8"], "k_fp8"), _ptr(k_scale, d["f32"], "k_scale"),
+        _ptr(q_pos0, d["i32"], "q_pos0"), _ptr(kv_len, d["i32"], "kv_len"),
+        int(row_begin), int(row_end), _ptr(scores, d["f32"], "scores"), _stream(stream)))
+
+
+def dsa_topk(shape, scores, row_begin, row_end, q_pos0, kv_len, indices, ws=None,
+             ws_bytes=0, stream=None):
+    d = _dt()
+    _raise(load_library().dsa_topk(
+        ctypes.byref(shape), _ptr(scores, d["f32"], "scores"), int(row_begin), int(row_end),
+        _ptr(q_pos0, d["i32"], "q_pos0"), _ptr(kv_len, d["i32"], "kv_len"),
+        _ptr(indices, d["i32"], "indices"), _ptr(ws, None, "ws"), int(ws_bytes),
+        _stream(stream)))
+
+
+def dsa_sparse_attn(shape, q, kv, indices, out, lse=None, ws=None, ws_bytes=0, stream=None):
+    import torch
+    d = _dt()
+    out_dtype = DSA_OUT_BF16 if out.dtype == torch.bfloat16 else DSA_OUT_F32
+    _raise(load_library().dsa_sparse_attn(
+        ctypes.byref(shape), _ptr(q, d["bf16"], "q"), _ptr(kv, d["bf16"], "kv"),
+        _ptr(indices, d["i32"], "indices"), _ptr(out, (torch.float32, torch.bfloat16), "out"),
+        out_dtype, _ptr(lse, d["f32"], "lse"), _ptr(ws, None, "ws"), int(ws_bytes),
+        _stream(stream)))
+
+
+def dsa_forward(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, q, kv,
+                indices_out, out, lse=None, ws=None, ws_bytes=0, stream=None):
+    import torch
+    d = _dt()
+    out_dtype = DSA_OUT_BF16 if out.dtype == torch.bfloat16 else DSA_OUT_F32
+    _raise(load_library().dsa_forward(
+        ctypes.byref(shape), _ptr(q_fp8, d["u8"], "q_fp8"), _ptr(q_scale, d["f32"], "q_scale"),
+        _ptr(w, d["f32"], "w"), _ptr(k_fp8, d["u8"], "k_fp8"), _ptr(k_scale, d["f32"], "k_scale"),
+        _ptr(q_pos0, d["i32"], "q_pos0"), _ptr(kv_len, d["i32"], "kv_len"),
+        _ptr(q, d["bf16"], "q"), _ptr(kv, d["bf16"], "kv"),
+        _ptr(indices_out, d["i32"], "indices_out"),
+        _ptr(out, (torch.float32, torch.bfloat16), "out"), out_dtype,
+        _ptr(lse, d["f32"], "lse"), _ptr(ws, None, "ws"), int(ws_bytes), _stream(stream)))
+
+
+def dsa_check(stream=None):
+    _raise(load_library().dsa_check(_stream(stream)))
+
+
+# ------------------------------------------------------------------ conveniences
+
+def alloc_workspace(shape: DsaShape, op: int, device="cuda"):
+    """A 256-byte aligned uint8 workspace tensor of the size ``op`` needs."""
+    import torch
+    n = workspace_size(shape, op)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device), n
+
+
+def forward(inp: dict, cfg: DsaConfig, out_dtype=None, ws=None, stream=None):
+    """Run the whole path on CUDA tensors from ``make_inputs``; returns
+    dict(indices, out, lse). Output buffers are allocated with torch."""
+    import torch
+    shape = shape_of(cfg)
+    dev = inp["q"].device
+    B, T = cfg.batch, cfg.n_q
+    out = torch.empty(B, T, cfg.heads, cfg.v_dim, device=dev,
+                      dtype=out_dtype or torch.float32)
+    lse = torch.empty(B, T, cfg.heads, device=dev, dtype=torch.float32)
+    idx = torch.empty(B, T, cfg.topk, device=dev, dtype=torch.int32)
+    if ws is None:
+        ws, n = alloc_workspace(shape, DSA_OP_FORWARD, dev)
+    else:
+        n = ws.numel()
+    dsa_forward(shape, inp["q_fp8"], inp["q_scale"], inp["w"], inp["k_fp8"], inp["k_scale"],
+                inp["q_pos0"], inp["kv_len"], inp["q"], inp["kv"], idx, out, lse, ws, n, stream)
+    return {"indices": idx, "out": out, "lse": lse}

@@ -1,0 +1,528 @@
+// Host side of the DSA C ABI (include/dsa.h): argument validation, tile
+// dispatch, TMA descriptor set-up and launches on the caller's stream.
+// One translation unit holds every kernel so the device error word is a
+// single symbol per device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstdarg>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/dsa.h"
+#include "indexer.cuh"
+#include "sparse_attn.cuh"
+#include "topk.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+dsa_status fail(dsa_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+dsa_status fail(dsa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+dsa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(DSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define DSA_CUDA_TRY(expr, what)                 \
+  do {                                           \
+    cudaError_t e_ = (expr);                     \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+constexpr int kNumSms = 148;
+constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------------------ device check
+
+dsa_status current_device(int* dev) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return fail(DSA_ERR_NO_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
+  if (*dev < 0 || *dev >= kMaxDevices) return fail(DSA_ERR_NO_DEVICE, "device ordinal out of range");
+  static int major[kMaxDevices] = {0};
+  if (major[*dev] == 0) {
+    int mj = 0;
+    cudaDeviceGetAttribute(&mj, cudaDevAttrComputeCapabilityMajor, *dev);
+    major[*dev] = mj;
+  }
+  if (major[*dev] != 10)
+    return fail(DSA_ERR_NO_DEVICE, "device %d is sm_%d0, this library is built for sm_100a", *dev,
+                major[*dev]);
+  return DSA_OK;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D byte tensor [rows, row_bytes] with a box of [box_rows, row_bytes] and the
+// swizzle that matches the row width (32, 64 or 128 bytes).
+dsa_status make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint32_t row_bytes,
+                        uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {row_bytes, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = row_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                  : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return DSA_OK;
+}
+
+// ------------------------------------------------------------------ validation
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+dsa_status check_shape_common(const dsa_shape* s) {
+  if (!s) return fail(DSA_ERR_INVALID_ARG, "shape is NULL");
+  if (s->batch < 1 || s->n_q < 1 || s->n_kv < 1)
+    return fail(DSA_ERR_INVALID_ARG, "batch, n_q and n_kv must be >= 1 (got %d, %d, %d)",
+                s->batch, s->n_q, s->n_kv);
+  if (static_cast<int64_t>(s->batch) * s->n_q > (1ll << 30) ||
+      static_cast<int64_t>(s->batch) * s->n_kv > (1ll << 30))
+    return fail(DSA_ERR_INVALID_ARG, "batch * rows exceeds 2^30");
+  return DSA_OK;
+}
+
+dsa_status check_indexer_shape(const dsa_shape* s) {
+  if (dsa_status st = check_shape_common(s)) return st;
+  const bool ok = (s->idx_heads == 64 && s->idx_dim == 128) || (s->idx_heads == 4 && s->idx_dim == 32);
+  if (!ok)
+    return fail(DSA_ERR_UNSUPPORTED, "indexer shape (H^I=%d, d^I=%d) is not compiled in; supported: (64,128), (4,32)",
+                s->idx_heads, s->idx_dim);
+  if (static_cast<int64_t>(s->batch) * s->n_q * s->idx_heads >= (1ll << 31))
+    return fail(DSA_ERR_INVALID_ARG, "batch * n_q * H^I exceeds the TMA coordinate range");
+  return DSA_OK;
+}
+
+dsa_status check_topk_shape(const dsa_shape* s) {
+  if (dsa_status st = check_shape_common(s)) return st;
+  if (s->topk < 1) return fail(DSA_ERR_INVALID_ARG, "topk must be >= 1 (got %d)", s->topk);
+  if (static_cast<int64_t>(s->batch) * s->n_q * s->topk >= (1ll << 40))
+    return fail(DSA_ERR_INVALID_ARG, "index array too large");
+  return DSA_OK;
+}
+
+dsa_status check_attn_shape(const dsa_shape* s) {
+  if (dsa_status st = check_topk_shape(s)) return st;
+  const bool big = s->qk_dim == 576 && s->v_dim == 512;
+  const bool tiny = s->qk_dim == 64 && s->v_dim == 64;
+  if (!big && !tiny)
+    return fail(DSA_ERR_UNSUPPORTED, "(qk_dim=%d, v_dim=%d) is not compiled in; supported: (576,512), (64,64)",
+                s->qk_dim, s->v_dim);
+  if (s->heads < 1 || s->heads > 128)
+    return fail(DSA_ERR_UNSUPPORTED, "heads must be in [1, 128] (got %d)", s->heads);
+  if (!(std::isfinite(s->softmax_scale)))
+    return fail(DSA_ERR_INVALID_ARG, "softmax_scale must be finite");
+  return DSA_OK;
+}
+
+// ------------------------------------------------------------------ kernel attributes
+
+template <class K>
+dsa_status set_smem(K kernel, int bytes, int dev, bool* done_flags) {
+  if (!done_flags[dev]) {
+    DSA_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+                 "cudaFuncSetAttribute");
+    done_flags[dev] = true;
+  }
+  return DSA_OK;
+}
+
+// ------------------------------------------------------------------ indexer launch
+
+template <int HI, int DI, int QG>
+dsa_status launch_indexer_t(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
+                            const float* w, const uint8_t* k_fp8, const float* k_scale,
+                            const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
+                            int32_t rows, float* scores, int write_invalid, cudaStream_t stream,
+                            int dev) {
+  using T = dsa::IndexerTile<HI, DI, QG>;
+  static bool attr_done[kMaxDevices] = {false};
+  if (dsa_status st = set_smem(dsa::indexer_scores_kernel<HI, DI, QG>, T::SMEM_BYTES, dev, attr_done))
+    return st;
+  CUtensorMap tq, tk;
+  if (dsa_status st = make_tmap_u8(&tq, q_fp8, static_cast<uint64_t>(s->batch) * s->n_q * HI, DI, T::N))
+    return st;
+  if (dsa_status st = make_tmap_u8(&tk, k_fp8, static_cast<uint64_t>(s->batch) * s->n_kv, DI, T::M))
+    return st;
+  dsa::IndexerParams p{};
+  p.q_scale = q_scale;
+  p.w = w;
+  p.k_scale = k_scale;
+  p.q_pos0 = q_pos0;
+  p.kv_len = kv_len;
+  p.scores = scores;
+  p.B = s->batch;
+  p.n_q = s->n_q;
+  p.n_kv = s->n_kv;
+  p.row_begin = row_begin;
+  p.rows = rows;
+  p.n_groups = (rows + QG - 1) / QG;
+  const int n_tiles = (s->n_kv + T::M - 1) / T::M;
+  const int64_t groups = static_cast<int64_t>(s->batch) * p.n_groups;
+  int64_t tps = (groups * n_tiles + 4 * kNumSms - 1) / (4 * kNumSms);
+  tps = std::max<int64_t>(4, std::min<int64_t>(tps, 64));
+  tps = std::min<int64_t>(tps, n_tiles);
+  p.tiles_per_split = static_cast<int32_t>(tps);
+  p.write_invalid = write_invalid;
+  const int n_splits = (n_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
+  if (p.n_groups > 65535 || s->batch > 65535)
+    return fail(DSA_ERR_INVALID_ARG, "row range too large for one indexer launch");
+  dim3 grid(n_splits, p.n_groups, s->batch);
+  dsa::indexer_scores_kernel<HI, DI, QG><<<grid, T::THREADS, T::SMEM_BYTES, stream>>>(tq, tk, p);
+  DSA_CUDA_TRY(cudaGetLastError(), "indexer launch");
+  return DSA_OK;
+}
+
+dsa_status launch_indexer(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
+                          const float* w, const uint8_t* k_fp8, const float* k_scale,
+                          const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
+                          int32_t rows, float* scores, int write_invalid, cudaStream_t stream,
+                          int dev) {
+  if (s->idx_heads == 64) {
+    if (rows == 1)
+      return launch_indexer_t<64, 128, 1>(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+                                          row_begin, rows, scores, write_invalid, stream, dev);
+    return launch_indexer_t<64, 128, 4>(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+                                        row_begin, rows, scores, write_invalid, stream, dev);
+  }
+  if (rows <= 4)
+    return launch_indexer_t<4, 32, 4>(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+                                      row_begin, rows, scores, write_invalid, stream, dev);
+  return launch_indexer_t<4, 32, 64>(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+                                     row_begin, rows, scores, write_invalid, stream, dev);
+}
+
+// ------------------------------------------------------------------ top-k launch
+
+dsa_status launch_topk(const dsa_shape* s, const float* scores, int32_t row_begin, int32_t rows,
+                       const int32_t* q_pos0, const int32_t* kv_len, int32_t* indices,
+                       int32_t out_rows, int32_t out_row0, cudaStream_t stream, int dev) {
+  static bool attr_done[kMaxDevices] = {false};
+  const int smem = dsa::kTopkSmemKeys * 4;
+  if (dsa_status st = set_smem(dsa::topk_kernel, smem, dev, attr_done)) return st;
+  if (s->batch > 65535) return fail(DSA_ERR_INVALID_ARG, "batch > 65535");
+  dsa::TopkParams p{};
+  p.scores = scores;
+  p.q_pos0 = q_pos0;
+  p.kv_len = kv_len;
+  p.indices = indices;
+  p.rows = rows;
+  p.row_begin = row_begin;
+  p.n_kv = s->n_kv;
+  p.k = s->topk;
+  p.out_rows = out_rows;
+  p.out_row0 = out_row0;
+  dim3 grid(rows, s->batch);
+  dsa::topk_kernel<<<grid, dsa::kTopkThreads, smem, stream>>>(p);
+  DSA_CUDA_TRY(cudaGetLastError(), "top-k launch");
+  return DSA_OK;
+}
+
+// ------------------------------------------------------------------ attention launch
+
+struct AttnPlan {
+  int vsplit, splits, slots_per_split;
+  size_t ws_bytes;
+};
+
+AttnPlan plan_attn(const dsa_shape* s) {
+  AttnPlan pl{};
+  pl.vsplit = s->qk_dim == 576 ? 2 : 1;
+  const int64_t rows = static_cast<int64_t>(s->batch) * s->n_q;
+  const int64_t ctas = rows * pl.vsplit;
+  const int max_splits = (s->topk + 31) / 32;
+  int splits = 1;
+  if (ctas < kNumSms / 2) {
+    splits = static_cast<int>(std::min<int64_t>(max_splits, (kNumSms + ctas - 1) / ctas));
+    splits = std::max(1, std::min(splits, 16));
+  }
+  int sps = (s->topk + splits - 1) / splits;
+  sps = (sps + 31) / 32 * 32;
+  splits = (s->topk + sps - 1) / sps;
+  pl.splits = splits;
+  pl.slots_per_split = sps;
+  pl.ws_bytes = 0;
+  if (splits > 1) {
+    const size_t po = static_cast<size_t>(rows) * splits * s->heads * s->v_dim * sizeof(float);
+    const size_t pl_ = static_cast<size_t>(rows) * splits * s->heads * sizeof(float);
+    pl.ws_bytes = (po + 255) / 256 * 256 + (pl_ + 255) / 256 * 256;
+  }
+  return pl;
+}
+
+template <int DQK, int DV, int VSPLIT>
+dsa_status launch_attn_t(const dsa_shape* s, const AttnPlan& pl, const uint16_t* q,
+                         const uint16_t* kv, const int32_t* indices, void* out, int out_bf16,
+                         float* lse, void* ws, cudaStream_t stream, int dev) {
+  using T = dsa::AttnTile<DQK, DV, VSPLIT>;
+  static bool attr_done[kMaxDevices] = {false};
+  if (dsa_status st = set_smem(dsa::sparse_attn_kernel<DQK, DV, VSPLIT>, T::SMEM_BYTES, dev, attr_done))
+    return st;
+  dsa::AttnParams p{};
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.kv = reinterpret_cast<const __nv_bfloat16*>(kv);
+  p.indices = indices;
+  p.out = out;
+  p.lse = lse;
+  p.B = s->batch;
+  p.n_q = s->n_q;
+  p.n_kv = s->n_kv;
+  p.topk = s->topk;
+  p.H = s->heads;
+  p.splits = pl.splits;
+  p.slots_per_split = pl.slots_per_split;
+  p.out_bf16 = out_bf16;
+  p.scale_log2 = s->softmax_scale * 1.4426950408889634f;
+  const int64_t rows = static_cast<int64_t>(s->batch) * s->n_q;
+  if (pl.splits > 1) {
+    const size_t po = static_cast<size_t>(rows) * pl.splits * s->heads * s->v_dim * sizeof(float);
+    p.part_o = static_cast<float*>(ws);
+    p.part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + (po + 255) / 256 * 256);
+  }
+  const int64_t nblocks = rows * pl.splits * VSPLIT;
+  if (nblocks >= (1ll << 31)) return fail(DSA_ERR_INVALID_ARG, "too many attention rows");
+  dsa::sparse_attn_kernel<DQK, DV, VSPLIT>
+      <<<static_cast<unsigned>(nblocks), T::THREADS, T::SMEM_BYTES, stream>>>(p);
+  DSA_CUDA_TRY(cudaGetLastError(), "sparse attention launch");
+  if (pl.splits > 1) {
+    if (rows > 0x7fffffffll) return fail(DSA_ERR_INVALID_ARG, "too many rows");
+    dim3 grid(static_cast<unsigned>(rows), s->heads);
+    dsa::attn_combine_kernel<<<grid, 128, 0, stream>>>(p, DV);
+    DSA_CUDA_TRY(cudaGetLastError(), "attention combine launch");
+  }
+  return DSA_OK;
+}
+
+dsa_status launch_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv,
+                       const int32_t* indices, void* out, int out_bf16, float* lse, void* ws,
+                       size_t ws_bytes, cudaStream_t stream, int dev) {
+  const AttnPlan pl = plan_attn(s);
+  if (pl.ws_bytes > 0) {
+    if (!ws || ws_bytes < pl.ws_bytes)
+      return fail(DSA_ERR_WORKSPACE, "attention needs %zu workspace bytes, got %zu", pl.ws_bytes,
+                  ws ? ws_bytes : size_t(0));
+    if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  }
+  if (s->qk_dim == 576)
+    return launch_attn_t<576, 512, 2>(s, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
+  return launch_attn_t<64, 64, 1>(s, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
+}
+
+// ------------------------------------------------------------------ forward plan
+
+struct FwdPlan {
+  int chunk_rows;
+  size_t scores_bytes, attn_bytes, total;
+};
+
+FwdPlan plan_forward(const dsa_shape* s) {
+  FwdPlan f{};
+  const size_t row_bytes = static_cast<size_t>(s->batch) * s->n_kv * sizeof(float);
+  const size_t budget = 256ull << 20;   // scores of one row chunk (L2-sized pieces at 64K+)
+  int64_t chunk = static_cast<int64_t>(budget / row_bytes);
+  chunk = std::max<int64_t>(chunk, 64);
+  chunk = std::min<int64_t>(chunk, s->n_q);
+  if (chunk < s->n_q) chunk = std::max<int64_t>(64, chunk / 64 * 64);
+  f.chunk_rows = static_cast<int>(chunk);
+  f.scores_bytes = (row_bytes * chunk + 255) / 256 * 256;
+  f.attn_bytes = plan_attn(s).ws_bytes;
+  f.total = f.scores_bytes + f.attn_bytes;
+  return f;
+}
+
+dsa_status check_ptrs(std::initializer_list<const void*> ptrs, const char* what) {
+  for (const void* p : ptrs)
+    if (!p) return fail(DSA_ERR_INVALID_ARG, "%s: required pointer is NULL", what);
+  return DSA_OK;
+}
+
+}  // namespace
+
+// ======================================================================== C ABI
+
+extern "C" {
+
+const char* dsa_version(void) { return "0.1.0"; }
+
+const char* dsa_status_string(dsa_status st) {
+  switch (st) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case DSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_TIMEOUT: return "device wait timed out";
+    case DSA_ERR_NO_DEVICE: return "no sm_100 device";
+  }
+  return "unknown status";
+}
+
+const char* dsa_last_error(void) { return g_last_error.c_str(); }
+
+dsa_status dsa_workspace_size(const dsa_shape* s, int32_t op, size_t* bytes) {
+  if (!bytes) return fail(DSA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = 0;
+  switch (op) {
+    case DSA_OP_INDEXER:
+      return check_indexer_shape(s);
+    case DSA_OP_TOPK:
+      return check_topk_shape(s);
+    case DSA_OP_SPARSE_ATTN: {
+      if (dsa_status st = check_attn_shape(s)) return st;
+      *bytes = plan_attn(s).ws_bytes;
+      return DSA_OK;
+    }
+    case DSA_OP_FORWARD: {
+      if (dsa_status st = check_indexer_shape(s)) return st;
+      if (dsa_status st = check_attn_shape(s)) return st;
+      *bytes = plan_forward(s).total;
+      return DSA_OK;
+    }
+    default:
+      return fail(DSA_ERR_INVALID_ARG, "unknown op %d", op);
+  }
+}
+
+dsa_status dsa_indexer_scores(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
+                              const float* w, const uint8_t* k_fp8, const float* k_scale,
+                              const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
+                              int32_t row_end, float* scores, void* stream) {
+  if (dsa_status st = check_indexer_shape(s)) return st;
+  if (dsa_status st = check_ptrs({q_fp8, q_scale, w, k_fp8, k_scale, scores}, "dsa_indexer_scores"))
+    return st;
+  if (row_begin < 0 || row_end > s->n_q || row_begin >= row_end)
+    return fail(DSA_ERR_INVALID_ARG, "row range [%d, %d) outside [0, %d) or empty", row_begin,
+                row_end, s->n_q);
+  if (!aligned(q_fp8, 16) || !aligned(k_fp8, 16))
+    return fail(DSA_ERR_INVALID_ARG, "q_fp8 and k_fp8 must be 16-byte aligned");
+  int dev;
+  if (dsa_status st = current_device(&dev)) return st;
+  return launch_indexer(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, row_begin,
+                        row_end - row_begin, scores, 1, static_cast<cudaStream_t>(stream), dev);
+}
+
+dsa_status dsa_topk(const dsa_shape* s, const float* scores, int32_t row_begin, int32_t row_end,
+                    const int32_t* q_pos0, const int32_t* kv_len, int32_t* indices, void* ws,
+                    size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (dsa_status st = check_topk_shape(s)) return st;
+  if (dsa_status st = check_ptrs({scores, indices}, "dsa_topk")) return st;
+  if (row_begin < 0 || row_end > s->n_q || row_begin >= row_end)
+    return fail(DSA_ERR_INVALID_ARG, "row range [%d, %d) outside [0, %d) or empty", row_begin,
+                row_end, s->n_q);
+  int dev;
+  if (dsa_status st = current_device(&dev)) return st;
+  return launch_topk(s, scores, row_begin, row_end - row_begin, q_pos0, kv_len, indices,
+                     row_end - row_begin, 0, static_cast<cudaStream_t>(stream), dev);
+}
+
+dsa_status dsa_sparse_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv,
+                           const int32_t* indices, void* out, int32_t out_dtype, float* lse,
+                           void* ws, size_t ws_bytes, void* stream) {
+  if (dsa_status st = check_attn_shape(s)) return st;
+  if (dsa_status st = check_ptrs({q, kv, indices, out}, "dsa_sparse_attn")) return st;
+  if (out_dtype != DSA_OUT_F32 && out_dtype != DSA_OUT_BF16)
+    return fail(DSA_ERR_INVALID_ARG, "out_dtype must be DSA_OUT_F32 or DSA_OUT_BF16");
+  if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16))
+    return fail(DSA_ERR_INVALID_ARG, "q, kv and out must be 16-byte aligned");
+  int dev;
+  if (dsa_status st = current_device(&dev)) return st;
+  return launch_attn(s, q, kv, indices, out, out_dtype == DSA_OUT_BF16, lse, ws, ws_bytes,
+                     static_cast<cudaStream_t>(stream), dev);
+}
+
+dsa_status dsa_forward(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
+                       const float* w, const uint8_t* k_fp8, const float* k_scale,
+                       const int32_t* q_pos0, const int32_t* kv_len, const uint16_t* q,
+                       const uint16_t* kv, int32_t* indices_out, void* out, int32_t out_dtype,
+                       float* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (dsa_status st = check_indexer_shape(s)) return st;
+  if (dsa_status st = check_attn_shape(s)) return st;
+  if (dsa_status st = check_ptrs({q_fp8, q_scale, w, k_fp8, k_scale, q, kv, indices_out, out},
+                                 "dsa_forward"))
+    return st;
+  if (out_dtype != DSA_OUT_F32 && out_dtype != DSA_OUT_BF16)
+    return fail(DSA_ERR_INVALID_ARG, "out_dtype must be DSA_OUT_F32 or DSA_OUT_BF16");
+  if (!aligned(q_fp8, 16) || !aligned(k_fp8, 16) || !aligned(q, 16) || !aligned(kv, 16) ||
+      !aligned(out, 16))
+    return fail(DSA_ERR_INVALID_ARG, "q_fp8, k_fp8, q, kv and out must be 16-byte aligned");
+  const FwdPlan f = plan_forward(s);
+  if (!ws || ws_bytes < f.total)
+    return fail(DSA_ERR_WORKSPACE, "dsa_forward needs %zu workspace bytes, got %zu", f.total,
+                ws ? ws_bytes : size_t(0));
+  if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  int dev;
+  if (dsa_status st = current_device(&dev)) return st;
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  float* scores = static_cast<float*>(ws);
+  void* attn_ws = static_cast<char*>(ws) + f.scores_bytes;
+  for (int r0 = 0; r0 < s->n_q; r0 += f.chunk_rows) {
+    const int rows = std::min(f.chunk_rows, s->n_q - r0);
+    if (dsa_status e = launch_indexer(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, r0,
+                                      rows, scores, 0, st_, dev))
+      return e;
+    // The chunk's selections go straight to their rows of indices_out.
+    if (dsa_status e = launch_topk(s, scores, r0, rows, q_pos0, kv_len, indices_out, s->n_q, r0,
+                                   st_, dev))
+      return e;
+  }
+  return launch_attn(s, q, kv, indices_out, out, out_dtype == DSA_OUT_BF16, lse, attn_ws,
+                     f.attn_bytes, st_, dev);
+}
+
+dsa_status dsa_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  unsigned int word = 0;
+  e = cudaMemcpyFromSymbol(&word, dsa::g_error_word, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (word) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(dsa::g_error_word, &zero, sizeof(zero));
+    if (word & dsa::kErrTimeout)
+      return fail(DSA_ERR_TIMEOUT, "a device-side wait exceeded its limit (error word 0x%x)", word);
+    return fail(DSA_ERR_CUDA, "device error word 0x%x", word);
+  }
+  return DSA_OK;
+}
+
+}  // extern "C"

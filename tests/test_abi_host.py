@@ -1,0 +1,131 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching a device. These
+run without a GPU (no kernel is launched)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_attention_long_fp8_b200 as dsa
+from sparse_attention_long_fp8_b200 import build as dsa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dsa_build.build()
+    return dsa.load_library()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_path_calls():
+    names = _declared_functions()
+    for n in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
+              "dsa_workspace_size", "dsa_check", "dsa_status_string", "dsa_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def _shape(**kw):
+    cfg = dsa.custom_config("prefill_4k", **kw) if kw else dsa.CONFIGS["prefill_4k"]
+    return dsa.shape_of(cfg)
+
+
+FAKE = 0x100000  # never dereferenced: validation fails before any launch
+
+
+def _call_indexer(lib, shape, rb=0, re_=16, ptrs=None):
+    p = ptrs or [FAKE] * 5
+    return lib.dsa_indexer_scores(ctypes.byref(shape) if shape is not None else None,
+                                  p[0], p[1], p[2], p[3], p[4], None, None, rb, re_, FAKE, None)
+
+
+def test_status_strings(lib):
+    for st in range(7):
+        assert lib.dsa_status_string(st)
+    assert lib.dsa_version().decode().count(".") == 2
+
+
+def test_null_shape_is_invalid(lib):
+    assert _call_indexer(lib, None) == dsa.DSA_ERR_INVALID_ARG
+    assert b"shape" in lib.dsa_last_error()
+
+
+def test_null_pointer_is_invalid(lib):
+    st = _call_indexer(lib, _shape(), ptrs=[FAKE, None, FAKE, FAKE, FAKE])
+    assert st == dsa.DSA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("rb,re_", [(-1, 4), (5, 5), (10, 4), (0, 4097)])
+def test_bad_row_range(lib, rb, re_):
+    assert _call_indexer(lib, _shape(), rb, re_) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_misaligned_fp8_pointer(lib):
+    st = _call_indexer(lib, _shape(), ptrs=[FAKE + 8, FAKE, FAKE, FAKE, FAKE])
+    assert st == dsa.DSA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw", [dict(idx_heads=32), dict(idx_dim=64), dict(idx_heads=4)])
+def test_unsupported_indexer_shape(lib, kw):
+    assert _call_indexer(lib, _shape(**kw)) == dsa.DSA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(topk=0), dsa.DSA_ERR_INVALID_ARG),
+    (dict(heads=129), dsa.DSA_ERR_UNSUPPORTED),
+    (dict(qk_dim=128), dsa.DSA_ERR_UNSUPPORTED),
+    (dict(v_dim=256), dsa.DSA_ERR_UNSUPPORTED),
+    (dict(n_q=0), dsa.DSA_ERR_INVALID_ARG),
+    (dict(batch=0), dsa.DSA_ERR_INVALID_ARG),
+])
+def test_attention_shape_checks(lib, kw, status):
+    shape = _shape(**kw)
+    n = ctypes.c_size_t(0)
+    assert lib.dsa_workspace_size(ctypes.byref(shape), dsa.DSA_OP_SPARSE_ATTN, ctypes.byref(n)) == status
+    st = lib.dsa_sparse_attn(ctypes.byref(shape), FAKE, FAKE, FAKE, FAKE, 0, None, None, 0, None)
+    assert st == status
+
+
+def test_bad_out_dtype_and_workspace(lib):
+    shape = _shape()
+    assert lib.dsa_sparse_attn(ctypes.byref(shape), FAKE, FAKE, FAKE, FAKE, 7, None, None, 0,
+                               None) == dsa.DSA_ERR_INVALID_ARG
+    st = lib.dsa_forward(ctypes.byref(shape), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE,
+                         FAKE, FAKE, FAKE, 0, None, None, 0, None)
+    assert st == dsa.DSA_ERR_WORKSPACE
+
+
+def test_workspace_sizes(lib):
+    # prefill at 4K: one score chunk of 4096 x 4096 fp32, no split-K partials
+    assert dsa.workspace_size(_shape(), dsa.DSA_OP_FORWARD) == 4096 * 4096 * 4
+    assert dsa.workspace_size(_shape(), dsa.DSA_OP_SPARSE_ATTN) == 0
+    assert dsa.workspace_size(_shape(), dsa.DSA_OP_TOPK) == 0
+    # 64K: scores are chunked (256 MB of rows at a time), never the full L x L
+    big = dsa.shape_of(dsa.CONFIGS["prefill_64k"])
+    assert dsa.workspace_size(big, dsa.DSA_OP_FORWARD) == 1024 * 65536 * 4
+    # a handful of rows: split-K partials are needed
+    few = _shape(n_q=4)
+    assert dsa.workspace_size(few, dsa.DSA_OP_SPARSE_ATTN) > 0
+    with pytest.raises(dsa.DsaError):
+        dsa.workspace_size(_shape(), 9)
+
+
+def test_valid_call_without_device_reports_no_device(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    st = _call_indexer(lib, _shape())
+    assert st == dsa.DSA_ERR_NO_DEVICE
