@@ -58,6 +58,8 @@ typedef enum {
 
 typedef enum { DSA_OUT_F32 = 0, DSA_OUT_BF16 = 1 } dsa_out_dtype;
 
+typedef enum { DSA_SCORES_ALL = 0, DSA_SCORES_VISIBLE_ONLY = 1 } dsa_scores_flags;
+
 typedef enum {
   DSA_OP_INDEXER = 0,
   DSA_OP_TOPK = 1,
@@ -84,7 +86,10 @@ typedef struct {
  *   w       [B, n_q, H^I] fp32 head weights
  *   k_fp8   [B, n_kv, d^I] e4m3fn codes         k_scale [B, n_kv] fp32
  *   rows [row_begin, row_end) of every sequence are scored:
- *   scores  [B, row_end-row_begin, n_kv] fp32; invisible keys get -inf.
+ *   scores  [B, row_end-row_begin, n_kv] fp32; invisible keys get -inf,
+ *           unless flags has DSA_SCORES_VISIBLE_ONLY: then only the visible
+ *           keys of each row are written (what dsa_topk reads) and the rest
+ *           of the buffer is left as it was.
  *   I[t,s] = k_scale[s] * sum_j (w[t,j] q_scale[t,j]) ReLU(q8[t,j] . k8[s]),
  *   the dot products exact-product / fp32-accumulated on the tensor cores.
  */
@@ -93,7 +98,7 @@ dsa_status dsa_indexer_scores(const dsa_shape* shape, const uint8_t* q_fp8,
                               const uint8_t* k_fp8, const float* k_scale,
                               const int32_t* q_pos0, const int32_t* kv_len,
                               int32_t row_begin, int32_t row_end,
-                              float* scores, void* stream);
+                              int32_t flags, float* scores, void* stream);
 
 /*
  * Top-k selection per score row (page "DeepseekV3.2 拆解", eq. u_t: keep the
@@ -145,6 +150,13 @@ dsa_status dsa_forward(const dsa_shape* shape, const uint8_t* q_fp8,
                        const uint16_t* q, const uint16_t* kv,
                        int32_t* indices_out, void* out, int32_t out_dtype,
                        float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Rows per indexer/top-k chunk that dsa_forward uses for this shape: the
+ * scores of `rows` query rows (rows * n_kv fp32 per sequence) are the only
+ * score storage, so the L x L matrix is never held at once. A caller that
+ * composes the path from the stage calls gets the same launches by scoring
+ * [r, r + rows) with DSA_SCORES_VISIBLE_ONLY and selecting from it. */
+dsa_status dsa_forward_chunk_rows(const dsa_shape* shape, int32_t* rows);
 
 /* Workspace bytes an op needs for this shape (0 if none). Returns status. */
 dsa_status dsa_workspace_size(const dsa_shape* shape, int32_t op,

@@ -27,6 +27,9 @@ DSA_ERR_NO_DEVICE = 6
 DSA_OUT_F32 = 0
 DSA_OUT_BF16 = 1
 
+DSA_SCORES_ALL = 0
+DSA_SCORES_VISIBLE_ONLY = 1
+
 DSA_OP_INDEXER = 0
 DSA_OP_TOPK = 1
 DSA_OP_SPARSE_ATTN = 2
@@ -66,18 +69,19 @@ def load_library(path: str | None = None):
     lib = ctypes.CDLL(path)
     P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     SP = ctypes.POINTER(DsaShape)
-    lib.dsa_indexer_scores.argtypes = [SP, P, P, P, P, P, P, P, I32, I32, P, P]
+    lib.dsa_indexer_scores.argtypes = [SP, P, P, P, P, P, P, P, I32, I32, I32, P, P]
     lib.dsa_topk.argtypes = [SP, P, I32, I32, P, P, P, P, SZ, P]
     lib.dsa_sparse_attn.argtypes = [SP, P, P, P, P, I32, P, P, SZ, P]
     lib.dsa_forward.argtypes = [SP, P, P, P, P, P, P, P, P, P, P, P, I32, P, P, SZ, P]
     lib.dsa_workspace_size.argtypes = [SP, I32, ctypes.POINTER(SZ)]
     lib.dsa_check.argtypes = [P]
+    lib.dsa_forward_chunk_rows.argtypes = [SP, ctypes.POINTER(I32)]
     lib.dsa_status_string.argtypes = [ctypes.c_int]
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_last_error.restype = ctypes.c_char_p
     lib.dsa_version.restype = ctypes.c_char_p
     for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
-               "dsa_workspace_size", "dsa_check"):
+               "dsa_workspace_size", "dsa_check", "dsa_forward_chunk_rows"):
         getattr(lib, fn).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -132,14 +136,21 @@ def workspace_size(shape: DsaShape, op: int) -> int:
     return n.value
 
 
+def forward_chunk_rows(shape: DsaShape) -> int:
+    n = ctypes.c_int32(0)
+    _raise(load_library().dsa_forward_chunk_rows(ctypes.byref(shape), ctypes.byref(n)))
+    return n.value
+
+
 def dsa_indexer_scores(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
-                       row_begin, row_end, scores, stream=None):
+                       row_begin, row_end, scores, stream=None, flags=DSA_SCORES_ALL):
     d = _dt()
     _raise(load_library().dsa_indexer_scores(
         ctypes.byref(shape), _ptr(q_fp8, d["u8"], "q_fp8"), _ptr(q_scale, d["f32"], "q_scale"),
         _ptr(w, d["f32"], "w"), _ptr(k_fp8, d["u8"], "k_fp8"), _ptr(k_scale, d["f32"], "k_scale"),
         _ptr(q_pos0, d["i32"], "q_pos0"), _ptr(kv_len, d["i32"], "kv_len"),
-        int(row_begin), int(row_end), _ptr(scores, d["f32"], "scores"), _stream(stream)))
+        int(row_begin), int(row_end), int(flags), _ptr(scores, d["f32"], "scores"),
+        _stream(stream)))
 
 
 def dsa_topk(shape, scores, row_begin, row_end, q_pos0, kv_len, indices, ws=None,

@@ -421,11 +421,21 @@ dsa_status dsa_workspace_size(const dsa_shape* s, int32_t op, size_t* bytes) {
   }
 }
 
+dsa_status dsa_forward_chunk_rows(const dsa_shape* s, int32_t* rows) {
+  if (!rows) return fail(DSA_ERR_INVALID_ARG, "rows is NULL");
+  if (dsa_status st = check_indexer_shape(s)) return st;
+  if (dsa_status st = check_attn_shape(s)) return st;
+  *rows = plan_forward(s).chunk_rows;
+  return DSA_OK;
+}
+
 dsa_status dsa_indexer_scores(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
                               const float* w, const uint8_t* k_fp8, const float* k_scale,
                               const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
-                              int32_t row_end, float* scores, void* stream) {
+                              int32_t row_end, int32_t flags, float* scores, void* stream) {
   if (dsa_status st = check_indexer_shape(s)) return st;
+  if (flags != DSA_SCORES_ALL && flags != DSA_SCORES_VISIBLE_ONLY)
+    return fail(DSA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   if (dsa_status st = check_ptrs({q_fp8, q_scale, w, k_fp8, k_scale, scores}, "dsa_indexer_scores"))
     return st;
   if (row_begin < 0 || row_end > s->n_q || row_begin >= row_end)
@@ -436,7 +446,8 @@ dsa_status dsa_indexer_scores(const dsa_shape* s, const uint8_t* q_fp8, const fl
   int dev;
   if (dsa_status st = current_device(&dev)) return st;
   return launch_indexer(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, row_begin,
-                        row_end - row_begin, scores, 1, static_cast<cudaStream_t>(stream), dev);
+                        row_end - row_begin, scores, flags == DSA_SCORES_ALL ? 1 : 0,
+                        static_cast<cudaStream_t>(stream), dev);
 }
 
 dsa_status dsa_topk(const dsa_shape* s, const float* scores, int32_t row_begin, int32_t row_end,

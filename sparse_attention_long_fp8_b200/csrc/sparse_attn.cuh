@@ -158,16 +158,14 @@ __global__ void __launch_bounds__(288, 1)
                                 : static_cast<const void*>(p.kv);
         cp_async_16(dst, src, valid ? 16u : 0u);
       }
+      // Block i is published as soon as its rows land: the MMA warp needs
+      // S(i) before it can issue PV(i-1), which is what frees the next stage.
       cp_async_commit();
-      if (i > 0) {
-        cp_async_wait<1>();
-        fence_proxy_async_smem();
-        mbar_arrive(&c_full[(i - 1) & 1]);
-      }
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(&c_full[st]);
     }
     cp_async_wait<0>();
-    fence_proxy_async_smem();
-    if (ok && n_blocks > 0) mbar_arrive(&c_full[(n_blocks - 1) & 1]);
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -218,7 +216,8 @@ __global__ void __launch_bounds__(288, 1)
     const int h = quarter * 32 + lane;                       // head row = TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     float m_used = -INFINITY;   // running max (log2 domain) the P values are relative to
-    float l = 0.f;
+    float l = 0.f;              // sum of the fp32 p: gives the LSE
+    float l_mma = 0.f;          // sum of the bf16-rounded p the PV MMA used: normalises O
     bool ok = true;
     for (int i = 0; i < n_blocks && ok; ++i) {
       const int sb = i & 1;
@@ -262,17 +261,19 @@ __global__ void __launch_bounds__(288, 1)
           }
           tmem_wait_st();
           l *= alpha;
+          l_mma *= alpha;
         }
       }
       m_used = m_new;
       uint32_t pk[16];
-      float lsum = 0.f;
+      float lsum = 0.f, lsum_mma = 0.f;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const float p0 = exp2f(z[2 * j] - m_used);
         const float p1 = exp2f(z[2 * j + 1] - m_used);
         const __nv_bfloat162 pb2 = __floats2bfloat162_rn(p0, p1);
-        lsum += __low2float(pb2) + __high2float(pb2);
+        lsum += p0 + p1;
+        lsum_mma += __low2float(pb2) + __high2float(pb2);
         pk[j] = *reinterpret_cast<const uint32_t*>(&pb2);
       }
       // empty block (no valid slot and no previous max): exp2(-inf - (-inf)) = NaN guard
@@ -280,8 +281,10 @@ __global__ void __launch_bounds__(288, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j) pk[j] = 0u;
         lsum = 0.f;
+        lsum_mma = 0.f;
       }
       l += lsum;
+      l_mma += lsum_mma;
       tmem_st16(tmem_base + lane_addr + T::COL_P + sb * (NK / 2), pk);
       tmem_wait_st();
       tc_fence_before();
@@ -292,8 +295,11 @@ __global__ void __launch_bounds__(288, 1)
       ok = mbar_wait(&pv_done[(n_blocks - 1) & 1], ((n_blocks - 1) >> 1) & 1);
       tc_fence_after();
     }
-    const bool has = ok && l > 0.f;
-    const float inv_l = has ? 1.0f / l : 0.f;
+    // O / sum(rounded p) is an exact convex combination of the V rows with
+    // weights perturbed by the bf16 rounding of p (a component shared by the
+    // rows cancels); the LSE keeps the unrounded sum.
+    const bool has = ok && l > 0.f && l_mma > 0.f;
+    const float inv_l = has ? 1.0f / l_mma : 0.f;
     const uint32_t keep = has ? 0xffffffffu : 0u;   // masks undefined TMEM when empty
     const float lse_v = has ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
     if (p.splits == 1) {

@@ -46,10 +46,11 @@ def _shape(**kw):
 FAKE = 0x100000  # never dereferenced: validation fails before any launch
 
 
-def _call_indexer(lib, shape, rb=0, re_=16, ptrs=None):
+def _call_indexer(lib, shape, rb=0, re_=16, ptrs=None, flags=0):
     p = ptrs or [FAKE] * 5
     return lib.dsa_indexer_scores(ctypes.byref(shape) if shape is not None else None,
-                                  p[0], p[1], p[2], p[3], p[4], None, None, rb, re_, FAKE, None)
+                                  p[0], p[1], p[2], p[3], p[4], None, None, rb, re_, flags,
+                                  FAKE, None)
 
 
 def test_status_strings(lib):
@@ -71,6 +72,10 @@ def test_null_pointer_is_invalid(lib):
 @pytest.mark.parametrize("rb,re_", [(-1, 4), (5, 5), (10, 4), (0, 4097)])
 def test_bad_row_range(lib, rb, re_):
     assert _call_indexer(lib, _shape(), rb, re_) == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_unknown_flags(lib):
+    assert _call_indexer(lib, _shape(), flags=2) == dsa.DSA_ERR_INVALID_ARG
 
 
 def test_misaligned_fp8_pointer(lib):
