@@ -138,6 +138,34 @@ dsa_status dsa_sparse_attn(const dsa_shape* shape, const uint16_t* q,
                            void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * dsa_sparse_attn without a caller-provided workspace. The paper has no
+ * counterpart: this entry point exists for callers that cannot call
+ * cudaMalloc - code whose device memory belongs to another framework's
+ * allocator, or a latency-critical decode loop that must not pay for (or
+ * synchronise on) an allocation - and so cannot hand in the split-K
+ * workspace that dsa_sparse_attn asks for when only a few query rows run.
+ *
+ * The split-K partials live in a static device array inside the library
+ * (16 MiB; every GPU that loads the library holds it until the process
+ * exits). Arguments, layouts and results are those of dsa_sparse_attn.
+ *   - Returns DSA_ERR_WORKSPACE, before any launch, when the shape's split-K
+ *     partials need more than 16 MiB (dsa_workspace_size(shape,
+ *     DSA_OP_SPARSE_ATTN) > 16 MiB); use dsa_sparse_attn for those.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first
+ *     call before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's
+ *     contents; each call writes every partial it reads, so nothing needs
+ *     clearing. Calls that overlap on the GPU (different streams, or other
+ *     host threads) race on it: serialise them.
+ *   - It allocates no device or host memory.
+ */
+dsa_status dsa_sparse_attn_noalloc(const dsa_shape* shape, const uint16_t* q,
+                                   const uint16_t* kv, const int32_t* indices,
+                                   void* out, int32_t out_dtype, float* lse,
+                                   void* stream);
+
+/*
  * The whole path for all n_q rows: indexer -> top-k -> sparse attention.
  *   Indexer inputs as dsa_indexer_scores, attention inputs as
  *   dsa_sparse_attn. indices_out [B, n_q, topk] receives the selection

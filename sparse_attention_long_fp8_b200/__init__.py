@@ -72,6 +72,7 @@ def load_library(path: str | None = None):
     lib.dsa_indexer_scores.argtypes = [SP, P, P, P, P, P, P, P, I32, I32, I32, P, P]
     lib.dsa_topk.argtypes = [SP, P, I32, I32, P, P, P, P, SZ, P]
     lib.dsa_sparse_attn.argtypes = [SP, P, P, P, P, I32, P, P, SZ, P]
+    lib.dsa_sparse_attn_noalloc.argtypes = [SP, P, P, P, P, I32, P, P]
     lib.dsa_forward.argtypes = [SP, P, P, P, P, P, P, P, P, P, P, P, I32, P, P, SZ, P]
     lib.dsa_workspace_size.argtypes = [SP, I32, ctypes.POINTER(SZ)]
     lib.dsa_check.argtypes = [P]
@@ -81,7 +82,8 @@ def load_library(path: str | None = None):
     lib.dsa_last_error.restype = ctypes.c_char_p
     lib.dsa_version.restype = ctypes.c_char_p
     for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
-               "dsa_workspace_size", "dsa_check", "dsa_forward_chunk_rows"):
+               "dsa_workspace_size", "dsa_check", "dsa_forward_chunk_rows",
+               "dsa_sparse_attn_noalloc"):
         getattr(lib, fn).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -172,6 +174,18 @@ def dsa_sparse_attn(shape, q, kv, indices, out, lse=None, ws=None, ws_bytes=0, s
         _ptr(indices, d["i32"], "indices"), _ptr(out, (torch.float32, torch.bfloat16), "out"),
         out_dtype, _ptr(lse, d["f32"], "lse"), _ptr(ws, None, "ws"), int(ws_bytes),
         _stream(stream)))
+
+
+def dsa_sparse_attn_noalloc(shape, q, kv, indices, out, lse=None, stream=None):
+    """dsa_sparse_attn for callers that cannot allocate: the split-K scratch
+    is a 16 MiB array inside the library (see include/dsa.h)."""
+    import torch
+    d = _dt()
+    out_dtype = DSA_OUT_BF16 if out.dtype == torch.bfloat16 else DSA_OUT_F32
+    _raise(load_library().dsa_sparse_attn_noalloc(
+        ctypes.byref(shape), _ptr(q, d["bf16"], "q"), _ptr(kv, d["bf16"], "kv"),
+        _ptr(indices, d["i32"], "indices"), _ptr(out, (torch.float32, torch.bfloat16), "out"),
+        out_dtype, _ptr(lse, d["f32"], "lse"), _stream(stream)))
 
 
 def dsa_forward(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, q, kv,

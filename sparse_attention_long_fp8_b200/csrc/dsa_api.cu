@@ -376,6 +376,32 @@ dsa_status check_ptrs(std::initializer_list<const void*> ptrs, const char* what)
 
 }  // namespace
 
+// ======================================================================== no-alloc scratch
+
+// Split-K partials of dsa_sparse_attn_noalloc. Host code may not use this
+// name as a device address: it is a host-side stand-in. The device address
+// comes from cudaGetSymbolAddress once per device.
+static constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on `dev` (the current device).
+dsa_status noalloc_scratch_addr(int dev, void** addr) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+    g_noalloc_addr[dev] = p;
+  }
+  *addr = g_noalloc_addr[dev];
+  return DSA_OK;
+}
+}  // namespace
+
 // ======================================================================== C ABI
 
 extern "C" {
@@ -478,6 +504,32 @@ dsa_status dsa_sparse_attn(const dsa_shape* s, const uint16_t* q, const uint16_t
   int dev;
   if (dsa_status st = current_device(&dev)) return st;
   return launch_attn(s, q, kv, indices, out, out_dtype == DSA_OUT_BF16, lse, ws, ws_bytes,
+                     static_cast<cudaStream_t>(stream), dev);
+}
+
+dsa_status dsa_sparse_attn_noalloc(const dsa_shape* s, const uint16_t* q, const uint16_t* kv,
+                                   const int32_t* indices, void* out, int32_t out_dtype,
+                                   float* lse, void* stream) {
+  if (dsa_status st = check_attn_shape(s)) return st;
+  if (dsa_status st = check_ptrs({q, kv, indices, out}, "dsa_sparse_attn_noalloc")) return st;
+  if (out_dtype != DSA_OUT_F32 && out_dtype != DSA_OUT_BF16)
+    return fail(DSA_ERR_INVALID_ARG, "out_dtype must be DSA_OUT_F32 or DSA_OUT_BF16");
+  if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16))
+    return fail(DSA_ERR_INVALID_ARG, "q, kv and out must be 16-byte aligned");
+  const AttnPlan pl = plan_attn(s);
+  if (pl.ws_bytes > kNoAllocScratchBytes)
+    return fail(DSA_ERR_WORKSPACE,
+                "this shape needs %zu bytes of split-K scratch; dsa_sparse_attn_noalloc holds at "
+                "most %zu (use dsa_sparse_attn with a workspace)",
+                pl.ws_bytes, kNoAllocScratchBytes);
+  int dev;
+  if (dsa_status st = current_device(&dev)) return st;
+  void* scratch = nullptr;
+  if (pl.ws_bytes > 0) {
+    if (dsa_status st = noalloc_scratch_addr(dev, &scratch)) return st;
+  }
+  return launch_attn(s, q, kv, indices, out, out_dtype == DSA_OUT_BF16, lse, scratch,
+                     pl.ws_bytes > 0 ? kNoAllocScratchBytes : 0,
                      static_cast<cudaStream_t>(stream), dev);
 }
 
