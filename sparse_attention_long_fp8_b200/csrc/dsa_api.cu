@@ -16,6 +16,7 @@
 #include "../../include/dsa.h"
 #include "indexer.cuh"
 #include "sparse_attn.cuh"
+#include "sparse_attn_pair.cuh"
 #include "topk.cuh"
 
 namespace {
@@ -236,7 +237,7 @@ dsa_status launch_topk(const dsa_shape* s, const float* scores, int32_t row_begi
                        const int32_t* q_pos0, const int32_t* kv_len, int32_t* indices,
                        int32_t out_rows, int32_t out_row0, cudaStream_t stream, int dev) {
   static bool attr_done[kMaxDevices] = {false};
-  const int smem = dsa::kTopkSmemKeys * 4;
+  const int smem = static_cast<int>(sizeof(dsa::TopkSmem));
   if (dsa_status st = set_smem(dsa::topk_kernel, smem, dev, attr_done)) return st;
   if (s->batch > 65535) return fail(DSA_ERR_INVALID_ARG, "batch > 65535");
   dsa::TopkParams p{};
@@ -331,6 +332,48 @@ dsa_status launch_attn_t(const dsa_shape* s, const AttnPlan& pl, const uint16_t*
   return DSA_OK;
 }
 
+// 576/512 latent: one 2-CTA cluster per (row, split), see sparse_attn_pair.cuh.
+dsa_status launch_attn_pair(const dsa_shape* s, const AttnPlan& pl, const uint16_t* q,
+                            const uint16_t* kv, const int32_t* indices, void* out, int out_bf16,
+                            float* lse, void* ws, cudaStream_t stream, int dev) {
+  using T = dsa::PairTile;
+  static bool attr_done[kMaxDevices] = {false};
+  if (dsa_status st = set_smem(dsa::sparse_attn_pair_kernel, T::SMEM_BYTES, dev, attr_done))
+    return st;
+  dsa::AttnParams p{};
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.kv = reinterpret_cast<const __nv_bfloat16*>(kv);
+  p.indices = indices;
+  p.out = out;
+  p.lse = lse;
+  p.B = s->batch;
+  p.n_q = s->n_q;
+  p.n_kv = s->n_kv;
+  p.topk = s->topk;
+  p.H = s->heads;
+  p.splits = pl.splits;
+  p.slots_per_split = pl.slots_per_split;
+  p.out_bf16 = out_bf16;
+  p.scale_log2 = s->softmax_scale * 1.4426950408889634f;
+  const int64_t rows = static_cast<int64_t>(s->batch) * s->n_q;
+  if (pl.splits > 1) {
+    const size_t po = static_cast<size_t>(rows) * pl.splits * s->heads * s->v_dim * sizeof(float);
+    p.part_o = static_cast<float*>(ws);
+    p.part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + (po + 255) / 256 * 256);
+  }
+  const int64_t nblocks = rows * pl.splits * 2;
+  if (nblocks >= (1ll << 31)) return fail(DSA_ERR_INVALID_ARG, "too many attention rows");
+  dsa::sparse_attn_pair_kernel<<<static_cast<unsigned>(nblocks), T::THREADS, T::SMEM_BYTES,
+                                 stream>>>(p);
+  DSA_CUDA_TRY(cudaGetLastError(), "sparse attention launch");
+  if (pl.splits > 1) {
+    dim3 grid(static_cast<unsigned>(rows), s->heads);
+    dsa::attn_combine_kernel<<<grid, 128, 0, stream>>>(p, s->v_dim);
+    DSA_CUDA_TRY(cudaGetLastError(), "attention combine launch");
+  }
+  return DSA_OK;
+}
+
 dsa_status launch_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv,
                        const int32_t* indices, void* out, int out_bf16, float* lse, void* ws,
                        size_t ws_bytes, cudaStream_t stream, int dev) {
@@ -342,7 +385,7 @@ dsa_status launch_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv
     if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   }
   if (s->qk_dim == 576)
-    return launch_attn_t<576, 512, 2>(s, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
+    return launch_attn_pair(s, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
   return launch_attn_t<64, 64, 1>(s, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
 }
 

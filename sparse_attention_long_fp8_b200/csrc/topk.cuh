@@ -3,12 +3,19 @@
 // score). Ties are broken by the lower key index.
 //
 // One CTA per score row. Scores are mapped to order-preserving uint32 keys
-// (larger float <=> larger key; -0 is folded into +0), then an MSB-first radix
-// select finds the exact k-th largest key u* in four 8-bit passes with shared
-// memory histograms. A final pass writes every key > u* and the lowest-index
-// keys == u* (an ordered block scan over the row, only when the ties at u*
-// do not all fit). Rows of up to kTopkSmemKeys visible scores are staged once in
-// shared memory; longer rows are re-read from global memory (L2) per pass.
+// (larger float <=> larger key; -0 is folded into +0).
+//   1. 1024 evenly spaced keys of the row are sorted (bitonic, shared
+//      memory) and a threshold tau is read off at about 1.25 k / n of the
+//      way down, so that roughly 1.25 k keys of the row are >= tau.
+//   2. One pass over the row appends every (key, index) with key >= tau to a
+//      candidate buffer in shared memory (warp-aggregated slots).
+//   3. If k <= #candidates <= capacity, an MSB-first radix select over the
+//      candidates finds the exact k-th key u*; every candidate above u* is
+//      written, then the lowest-index candidates equal to u*.
+//   Otherwise (a sample that missed, or many exact ties) the same radix
+//   select runs over the whole row, re-read from global memory per pass.
+// The result never depends on the sample: it only decides how much of the
+// row the exact select has to look at.
 #pragma once
 
 #include "ptx.cuh"
@@ -25,67 +32,55 @@ struct TopkParams {
 };
 
 constexpr int kTopkThreads = 1024;
-constexpr int kTopkSmemKeys = 48 * 1024;   // 192 KB of staged keys
+constexpr int kTopkSamples = 1024;
+constexpr int kTopkCap = 4096;      // candidate buffer (keys + indices: 32 KB)
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f + 0.0f);   // -0 -> +0
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
-  extern __shared__ __align__(16) uint32_t tk_smem[];
-  uint32_t* staged = tk_smem;                       // [kTopkSmemKeys]
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t s_sel_bin, s_above, s_count;
-  __shared__ uint32_t warp_tot[kTopkThreads / 32];
+struct TopkSmem {
+  uint32_t cand_u[kTopkCap];
+  int32_t cand_i[kTopkCap];
+  uint32_t samp[kTopkSamples];
+  uint32_t hist[256];
+  uint32_t warp_tot[kTopkThreads / 32];
+  uint32_t sel_bin, above, count, n_cand;
+};
 
-  const int r = blockIdx.x, b = blockIdx.y;
+// Exact k-th largest key among `n` keys given by get(i) (all threads of the
+// CTA call this). Returns u*; *need_out = number of keys equal to u* that
+// belong to the top k; *eq_out = number of keys equal to u*.
+template <class Get>
+__device__ uint32_t radix_kth(TopkSmem& sm, int n, uint32_t k, Get get, uint32_t* need_out,
+                              uint32_t* eq_out) {
   const int tid = threadIdx.x;
-  const int pos = (p.q_pos0 ? p.q_pos0[b] : 0) + p.row_begin + r;
-  const int kvl = min(p.kv_len ? p.kv_len[b] : p.n_kv, p.n_kv);
-  const int n = max(0, min(pos + 1, kvl));
-  const float* row = p.scores + (static_cast<size_t>(b) * p.rows + r) * p.n_kv;
-  int32_t* out = p.indices + (static_cast<size_t>(b) * p.out_rows + p.out_row0 + r) * p.k;
-
-  if (n <= p.k) {
-    for (int i = tid; i < p.k; i += kTopkThreads) out[i] = i < n ? i : -1;
-    return;
-  }
-  const bool use_smem = n <= kTopkSmemKeys;
-  if (use_smem) {
-    for (int i = tid; i < n; i += kTopkThreads) staged[i] = order_key(row[i]);
-    __syncthreads();
-  }
-
-  uint32_t prefix = 0, mask = 0;
-  uint32_t need = static_cast<uint32_t>(p.k);   // still to take among keys matching prefix
-  uint32_t eq_count = 0;
+  uint32_t prefix = 0, mask = 0, need = k, eq_count = 0;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
+    for (int i = tid; i < 256; i += kTopkThreads) sm.hist[i] = 0;
     __syncthreads();
     for (int c0 = 0; c0 < n; c0 += kTopkThreads) {
-      // Warp-aggregated increments: score keys cluster in few high bins, so
-      // lanes with the same bin merge into one atomic.
       const int i = c0 + tid;
       uint32_t bin = 256u;
       if (i < n) {
-        const uint32_t u = use_smem ? staged[i] : order_key(row[i]);
+        const uint32_t u = get(i);
         if ((u & mask) == prefix) bin = (u >> shift) & 255u;
       }
+      // lanes with the same bin merge into one atomic (keys cluster in few bins)
       const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (bin < 256u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+      if (bin < 256u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], __popc(peers));
     }
     __syncthreads();
     if (tid < 32) {
-      // lane l owns bins [248 - 8l, 255 - 8l] (high bins first)
       uint32_t c[8], sum = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        c[j] = hist[255 - (tid * 8 + j)];
+        c[j] = sm.hist[255 - (tid * 8 + j)];
         sum += c[j];
       }
-      uint32_t incl = sum;   // inclusive prefix over lanes (from the top)
+      uint32_t incl = sum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -97,55 +92,154 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           if (acc < need && need <= acc + c[j]) {
-            s_sel_bin = 255u - (tid * 8 + j);
-            s_above = acc;
-            s_count = c[j];
+            sm.sel_bin = 255u - (tid * 8 + j);
+            sm.above = acc;
+            sm.count = c[j];
           }
           acc += c[j];
         }
       }
     }
     __syncthreads();
-    const uint32_t bin = s_sel_bin;
-    need -= s_above;
-    eq_count = s_count;
-    prefix |= bin << shift;
+    need -= sm.above;
+    eq_count = sm.count;
+    prefix |= sm.sel_bin << shift;
     mask |= 255u << shift;
     __syncthreads();
   }
-  // prefix is now the exact k-th largest key u*; `need` keys equal to u* are
-  // taken (1 <= need <= eq_count) after every key > u*.
-  const uint32_t kth = prefix;
-  if (tid == 0) s_count = 0;
+  *need_out = need;
+  *eq_out = eq_count;
+  return prefix;
+}
+
+__global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
+  extern __shared__ __align__(16) uint8_t tk_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_raw);
+
+  const int r = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int pos = (p.q_pos0 ? p.q_pos0[b] : 0) + p.row_begin + r;
+  const int kvl = min(p.kv_len ? p.kv_len[b] : p.n_kv, p.n_kv);
+  const int n = max(0, min(pos + 1, kvl));
+  const float* row = p.scores + (static_cast<size_t>(b) * p.rows + r) * p.n_kv;
+  int32_t* out = p.indices + (static_cast<size_t>(b) * p.out_rows + p.out_row0 + r) * p.k;
+  const uint32_t k = static_cast<uint32_t>(p.k);
+
+  if (n <= p.k) {
+    for (int i = tid; i < p.k; i += kTopkThreads) out[i] = i < n ? i : -1;
+    return;
+  }
+
+  // ---- 1. threshold from a sorted sample (descending)
+  sm.samp[tid] = order_key(row[static_cast<int>((static_cast<int64_t>(tid) * n) / kTopkSamples)]);
+  if (tid == 0) sm.n_cand = 0;
+  __syncthreads();
+  for (int size = 2; size <= kTopkSamples; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const int j = tid ^ stride;
+      if (j > tid) {
+        const uint32_t a = sm.samp[tid], c = sm.samp[j];
+        const bool desc = (tid & size) == 0;
+        if (desc ? (a < c) : (a > c)) {
+          sm.samp[tid] = c;
+          sm.samp[j] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  const int64_t want =
+      (static_cast<int64_t>(5) * p.k * kTopkSamples) / (4 * static_cast<int64_t>(n)) + 8;
+  const uint32_t tau = sm.samp[want < kTopkSamples - 1 ? want : kTopkSamples - 1];
+
+  // ---- 2. one pass: candidates >= tau
+  for (int c0 = 0; c0 < n; c0 += kTopkThreads) {
+    const int i = c0 + tid;
+    const uint32_t u = i < n ? order_key(row[i]) : 0u;
+    const bool take = i < n && u >= tau;
+    const uint32_t bal = __ballot_sync(0xffffffffu, take);
+    uint32_t base = 0;
+    if (lane == 0 && bal) base = atomicAdd(&sm.n_cand, static_cast<uint32_t>(__popc(bal)));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    const uint32_t slot = base + __popc(bal & ((1u << lane) - 1u));
+    if (take && slot < static_cast<uint32_t>(kTopkCap)) {
+      sm.cand_u[slot] = u;
+      sm.cand_i[slot] = i;
+    }
+  }
+  __syncthreads();
+  const uint32_t n_cand = sm.n_cand;
+  __syncthreads();
+
+  if (n_cand >= k && n_cand <= static_cast<uint32_t>(kTopkCap)) {
+    // ---- 3. exact select among the candidates
+    uint32_t need, eq_count;
+    const uint32_t kth = radix_kth(sm, static_cast<int>(n_cand), k,
+                                   [&](int i) { return sm.cand_u[i]; }, &need, &eq_count);
+    if (tid == 0) sm.count = 0;
+    __syncthreads();
+    const bool take_all_eq = need == eq_count;
+    for (int c0 = 0; c0 < static_cast<int>(n_cand); c0 += kTopkThreads) {
+      const int i = c0 + tid;
+      const bool take = i < static_cast<int>(n_cand) &&
+                        (sm.cand_u[i] > kth || (take_all_eq && sm.cand_u[i] == kth));
+      const uint32_t bal = __ballot_sync(0xffffffffu, take);
+      uint32_t base = 0;
+      if (lane == 0 && bal) base = atomicAdd(&sm.count, static_cast<uint32_t>(__popc(bal)));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (take) out[base + __popc(bal & ((1u << lane) - 1u))] = sm.cand_i[i];
+    }
+    if (!take_all_eq) {
+      // ties at u*: a tied candidate is taken iff fewer than `need` tied
+      // candidates have a lower key index.
+      __syncthreads();
+      const uint32_t base_slot = sm.count;
+      for (int i = tid; i < static_cast<int>(n_cand); i += kTopkThreads) {
+        if (sm.cand_u[i] != kth) continue;
+        const int my = sm.cand_i[i];
+        uint32_t lower = 0;
+        for (int j = 0; j < static_cast<int>(n_cand); ++j)
+          lower += (sm.cand_u[j] == kth && sm.cand_i[j] < my) ? 1u : 0u;
+        if (lower < need) out[base_slot + lower] = my;
+      }
+    }
+    return;
+  }
+
+  // ---- fallback: exact select over the whole row (global memory per pass)
+  uint32_t need, eq_count;
+  const uint32_t kth = radix_kth(sm, n, k, [&](int i) { return order_key(row[i]); }, &need,
+                                 &eq_count);
+  if (tid == 0) sm.count = 0;
   __syncthreads();
   const bool take_all_eq = need == eq_count;
   for (int c0 = 0; c0 < n; c0 += kTopkThreads) {
     const int i = c0 + tid;
     bool take = false;
     if (i < n) {
-      const uint32_t u = use_smem ? staged[i] : order_key(row[i]);
+      const uint32_t u = order_key(row[i]);
       take = u > kth || (take_all_eq && u == kth);
     }
     const uint32_t bal = __ballot_sync(0xffffffffu, take);
     uint32_t base = 0;
-    if ((tid & 31) == 0 && bal) base = atomicAdd(&s_count, static_cast<uint32_t>(__popc(bal)));
+    if (lane == 0 && bal) base = atomicAdd(&sm.count, static_cast<uint32_t>(__popc(bal)));
     base = __shfl_sync(0xffffffffu, base, 0);
-    if (take) out[base + __popc(bal & ((1u << (tid & 31)) - 1u))] = i;
+    if (take) out[base + __popc(bal & ((1u << lane) - 1u))] = i;
   }
   if (!take_all_eq) {
+    // ordered block scan over the row: the first `need` keys equal to u*
     __syncthreads();
-    const uint32_t base_slot = s_count;   // = k - need
+    const uint32_t base_slot = sm.count;
     uint32_t taken = 0;
-    const int lane = tid & 31, w = tid >> 5;
     for (int c0 = 0; c0 < n && taken < need; c0 += kTopkThreads) {
       const int i = c0 + tid;
-      const bool eq = i < n && (use_smem ? staged[i] : order_key(row[i])) == kth;
+      const bool eq = i < n && order_key(row[i]) == kth;
       const uint32_t bal = __ballot_sync(0xffffffffu, eq);
-      if (lane == 0) warp_tot[w] = __popc(bal);
+      if (lane == 0) sm.warp_tot[w] = __popc(bal);
       __syncthreads();
       uint32_t before = 0, total = 0;
       for (int j = 0; j < kTopkThreads / 32; ++j) {
-        const uint32_t v = warp_tot[j];
+        const uint32_t v = sm.warp_tot[j];
         if (j < w) before += v;
         total += v;
       }
