@@ -306,6 +306,14 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
                : "memory");
 }
 
+// Relaxed remote arrive: orders nothing, so it does not wait for this
+// thread's earlier stores (st.async included) to land. Use it only to signal
+// that values this thread already consumed may be overwritten.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
+               : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx_u32(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");

@@ -264,10 +264,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
     };
     int idx_next = load_idx(0);
 
-    // A(i): read this CTA's partial logits of block i (32 keys) and send them
-    // to the peer.
-    auto stage_a = [&](int i, uint32_t (&sr)[32], uint32_t& vmask) -> bool {
-      const int xb = i & 1;
+    // Per block i the softmax warps run four steps:
+    //   load(i)  this CTA's partial logits (32 keys) from TMEM, free the S tile;
+    //   send(i)  those partials to the peer (st.async into its x buffer);
+    //   max(i)   add the peer's partials, block max over the 64 keys (shared
+    //            with the partner warp of the same lane quarter);
+    //   soft(i)  online softmax, P(i) into TMEM, hand the block to PV.
+    // They are interleaved as load(i+1), max(i), soft(i), send(i+1): block
+    // i+1's partials travel while the next S tile is computed, and the
+    // release-ordered arrives of max(i) and soft(i) (row-max hand-off, P
+    // ready) are not queued behind in-flight DSMEM stores.
+    auto load_s = [&](int i, uint32_t (&sr)[32], uint32_t& vmask) -> bool {
       const int idx = idx_next;
       idx_next = load_idx(i + 1);
       vmask = __ballot_sync(0xffffffffu, idx >= 0 && idx < p.n_kv);
@@ -278,6 +285,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
+      return true;
+    };
+    auto send_s = [&](int i, const uint32_t (&sr)[32]) -> bool {
+      const int xb = i & 1;
       if (expect_thread)
         mbar_arrive_expect_tx_u32(smem_u32(&x_full[xb]), static_cast<uint32_t>(T::X_BYTES));
       if (!mbar_wait(&x_free[xb], ((i >> 1) & 1) ^ 1)) return false;
@@ -290,13 +301,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       }
       return true;
     };
-
-    // B(i): add the peer's partial, online softmax over the block's 64 keys
-    // (row max shared with the partner warp), this warp's 32 p into TMEM.
-    auto stage_b = [&](int i, const uint32_t (&sr)[32], uint32_t vmask) -> bool {
+    auto block_max = [&](int i, const uint32_t (&sr)[32], uint32_t vmask, float (&z)[32],
+                         float& bmax) -> bool {
       const int xb = i & 1;
       if (!mbar_wait(&x_full[xb], (i >> 1) & 1)) return false;
-      float z[32];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int chunk = half * 8 + j;
@@ -304,9 +312,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
                                                           ((chunk ^ (h & 7)) << 4));
         z[4 * j] = f.x; z[4 * j + 1] = f.y; z[4 * j + 2] = f.z; z[4 * j + 3] = f.w;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(x_free_peer + xb * 8);
-
       float hmax = -INFINITY;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
@@ -316,6 +321,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
         z[j] = ((vmask >> j) & 1u) ? s * p.scale_log2 : -INFINITY;
         hmax = fmaxf(hmax, z[j]);
       }
+      // The peer's values are consumed (z depends on them): its x buffer
+      // slot may be reused.
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote_relaxed(x_free_peer + xb * 8);
       // row max over both halves of the block
       float* red_i = red + (i & 1) * (2 * T::M);
       red_i[half * T::M + h] = hmax;
@@ -323,7 +332,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
       uint64_t* rb = &red_bar[(i & 1) * 4 + quarter];
       if (lane == 0) mbar_arrive(rb);
       if (!mbar_wait(rb, (i >> 1) & 1)) return false;
-      const float bmax = fmaxf(hmax, red_i[(half ^ 1) * T::M + h]);
+      bmax = fmaxf(hmax, red_i[(half ^ 1) * T::M + h]);
+      return true;
+    };
+    auto softmax_p = [&](int i, const float (&z)[32], float bmax) -> bool {
       const bool grow = bmax > m_used + 8.0f;
       const float m_new = grow ? bmax : m_used;
       // The P tile and O are free once PV(i-1) finished.
@@ -376,15 +388,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(448, 1)
 
     uint32_t sr_a[32], sr_b[32];
     uint32_t vm_a = 0, vm_b = 0;
-    if (n_blocks > 0) ok = stage_a(0, sr_a, vm_a);
+    float z[32];
+    float bmax = -INFINITY;
+    if (n_blocks > 0) ok = load_s(0, sr_a, vm_a) && send_s(0, sr_a);
     for (int i = 0; i < n_blocks && ok; i += 2) {
-      if (i + 1 < n_blocks) ok = stage_a(i + 1, sr_b, vm_b);
-      if (!ok) break;
-      ok = stage_b(i, sr_a, vm_a);
+      if (i + 1 < n_blocks) ok = load_s(i + 1, sr_b, vm_b);
+      ok = ok && block_max(i, sr_a, vm_a, z, bmax);
+      ok = ok && softmax_p(i, z, bmax);
+      if (ok && i + 1 < n_blocks) ok = send_s(i + 1, sr_b);
       if (!ok || i + 1 >= n_blocks) break;
-      if (i + 2 < n_blocks) ok = stage_a(i + 2, sr_a, vm_a);
-      if (!ok) break;
-      ok = stage_b(i + 1, sr_b, vm_b);
+      if (i + 2 < n_blocks) ok = load_s(i + 2, sr_a, vm_a);
+      ok = ok && block_max(i + 1, sr_b, vm_b, z, bmax);
+      ok = ok && softmax_p(i + 1, z, bmax);
+      if (ok && i + 2 < n_blocks) ok = send_s(i + 2, sr_a);
     }
     if (ok && n_blocks > 0) {
       ok = mbar_wait(pv_done, (n_blocks - 1) & 1);
