@@ -16,7 +16,7 @@
 #include "../../include/dsa.h"
 #include "indexer.cuh"
 #include "sparse_attn.cuh"
-#include "sparse_attn_pair.cuh"
+#include "sparse_attn_vh.cuh"
 #include "topk.cuh"
 
 namespace {
@@ -332,13 +332,13 @@ dsa_status launch_attn_t(const dsa_shape* s, const AttnPlan& pl, const uint16_t*
   return DSA_OK;
 }
 
-// 576/512 latent: one 2-CTA cluster per (row, split), see sparse_attn_pair.cuh.
-dsa_status launch_attn_pair(const dsa_shape* s, const AttnPlan& pl, const uint16_t* q,
+// 576/512 latent: two CTAs per (row, split), one per value half, see sparse_attn_vh.cuh.
+dsa_status launch_attn_vh(const dsa_shape* s, const AttnPlan& pl, const uint16_t* q,
                             const uint16_t* kv, const int32_t* indices, void* out, int out_bf16,
                             float* lse, void* ws, cudaStream_t stream, int dev) {
-  using T = dsa::PairTile;
+  using T = dsa::VhTile;
   static bool attr_done[kMaxDevices] = {false};
-  if (dsa_status st = set_smem(dsa::sparse_attn_pair_kernel, T::SMEM_BYTES, dev, attr_done))
+  if (dsa_status st = set_smem(dsa::sparse_attn_vh_kernel, T::SMEM_BYTES, dev, attr_done))
     return st;
   dsa::AttnParams p{};
   p.q = reinterpret_cast<const __nv_bfloat16*>(q);
@@ -363,8 +363,8 @@ dsa_status launch_attn_pair(const dsa_shape* s, const AttnPlan& pl, const uint16
   }
   const int64_t nblocks = rows * pl.splits * 2;
   if (nblocks >= (1ll << 31)) return fail(DSA_ERR_INVALID_ARG, "too many attention rows");
-  dsa::sparse_attn_pair_kernel<<<static_cast<unsigned>(nblocks), T::THREADS, T::SMEM_BYTES,
-                                 stream>>>(p);
+  dsa::sparse_attn_vh_kernel<<<static_cast<unsigned>(nblocks), T::THREADS, T::SMEM_BYTES, stream>>>(
+      p);
   DSA_CUDA_TRY(cudaGetLastError(), "sparse attention launch");
   if (pl.splits > 1) {
     dim3 grid(static_cast<unsigned>(rows), s->heads);
@@ -385,7 +385,7 @@ dsa_status launch_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv
     if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   }
   if (s->qk_dim == 576)
-    return launch_attn_pair(s, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
+    return launch_attn_vh(s, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
   return launch_attn_t<64, 64, 1>(s, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
 }
 

@@ -1,0 +1,445 @@
+// Sparse MQA attention over the selected 576-d latent rows (page "DeepseekV3.2
+// 拆解", section "核心组件 / 细粒度 Token 选择机制", eq. u_t; latent = 512 value
+// dims + 64 RoPE dims, page "DeepSeek architecture", section 1.1).
+//
+// Two independent CTAs per query row, one per half of the 512 value dims
+// ("V-half" v = 0, 1). Each CTA
+//   * gathers the full 1152-byte latent rows of the selected keys into a
+//     2-stage ring of 64-key blocks (cp.async, completion on mbarriers);
+//   * computes the complete logits S = Q C^T (128 heads x 64 keys per block):
+//     Q's five 64-dim blocks that only the logits use live in TMEM (A operand
+//     read from TMEM), its four V-half blocks in shared memory;
+//   * runs the online softmax and accumulates O for its 256 value dims.
+// The logits are computed twice per row (once per CTA) and the rows gathered
+// twice (L2 serves the second read); in exchange no partial result crosses
+// between SMs: on this part DSMEM stores move ~11 bytes per cycle per SM,
+// which made a per-block exchange of fp32 partial logits the bound.
+//
+// A stage is released in two parts: its five logit-only dim blocks as soon as
+// S of the block completes, its four V-half blocks when PV completes. The
+// logit MMAs of a block run over the logit-only part first, so the gather of
+// block i + 2 overlaps S(i + 1) and PV(i).
+//
+// TMEM per CTA: O 256 columns, S 64, P 32, Q 160 = 512.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include <type_traits>
+
+#include "ptx.cuh"
+#include "sparse_attn.cuh"
+
+namespace dsa {
+
+struct VhTile {
+  static constexpr int NK = 64;                 // latent rows per block
+  static constexpr int M = 128;                 // head rows
+  static constexpr int DQK = 576, DV = 512, VH = 256;
+  static constexpr int NDB = DQK / 64;          // 9 dim blocks per latent row
+  static constexpr int VDB = VH / 64;           // 4 of them hold this CTA's value half
+  static constexpr int XDB = NDB - VDB;         // 5 only the logits read
+  static constexpr int DB_BYTES = NK * 128;     // one 64-dim block of a stage
+  static constexpr int STAGE_BYTES = NDB * DB_BYTES;
+  static constexpr int STAGES = 2;
+  static constexpr int QS_BYTES = VDB * M * 128;
+  static constexpr int PRODUCERS = 128;
+  static constexpr int THREADS = 448;           // gather 0-3, S MMA 4, softmax 5-12, PV MMA 13
+  static constexpr int SOFTMAX_WARPS = 8;       // two per TMEM lane quarter, 32 keys each
+  static constexpr int COL_O = 0, COL_S = 256, COL_P = 320, COL_Q = 352;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int OFF_C = 0;
+  static constexpr int OFF_QS = STAGES * STAGE_BYTES;
+  static constexpr int OFF_IDX = OFF_QS + QS_BYTES;          // [gather warp][NK] int32
+  static constexpr int OFF_RED = OFF_IDX + 4 * NK * 4;       // [2 parity][2 halves][128] fp32
+  static constexpr int OFF_END = OFF_RED + 2 * 2 * M * 4;    // [half][l, l_mma][128] fp32
+  static constexpr int OFF_BAR = OFF_END + 2 * 2 * M * 4;
+  static constexpr int NUM_BARS = 4 * STAGES + 5 + 8 + 4;    // stages, singles, red[8], end[4]
+  static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+  static_assert(STAGE_BYTES % 1024 == 0 && OFF_QS % 1024 == 0, "1024-byte aligned operands");
+  static_assert(COL_Q + XDB * 32 == 512, "TMEM columns");
+};
+
+// Latent dim block of the t-th logit-only block of V-half v (t = 0..4): the
+// other half's four value blocks, then the RoPE block 8.
+__device__ __forceinline__ int vh_xblock(int t, int v) { return t == 4 ? 8 : t + 4 * (1 - v); }
+
+// Warp roles: 0-3 gather (cp.async, 16 bytes per thread and copy); 4 issues
+// the logit MMAs and owns TMEM; 5-12 run the softmax (two warps per TMEM lane
+// quarter: a thread owns one head row and 32 of a block's 64 keys); 13 issues
+// the PV MMAs.
+__global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
+  using T = VhTile;
+  constexpr int NK = T::NK;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* c_smem = smem + T::OFF_C;
+  uint8_t* qs_smem = smem + T::OFF_QS;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::OFF_BAR);
+  uint64_t* cx_full = bars;                      // [2] logit-only blocks of the stage landed
+  uint64_t* cv_full = bars + T::STAGES;          // [2] V-half blocks landed
+  uint64_t* cx_empty = bars + 2 * T::STAGES;     // [2] S of the stage's block finished
+  uint64_t* cv_empty = bars + 3 * T::STAGES;     // [2] PV of the stage's block finished
+  uint64_t* s_full = bars + 4 * T::STAGES;       // S tile written
+  uint64_t* s_free = s_full + 1;                 // S tile read by the softmax warps
+  uint64_t* p_full = s_full + 2;                 // P tile written
+  uint64_t* pv_done = s_full + 3;                // PV finished (P tile free, O updated)
+  uint64_t* q_ready = s_full + 4;                // Q in TMEM and shared memory
+  uint64_t* red_bar = s_full + 5;                // [parity][quarter]: both half maxima written
+  uint64_t* end_bar = s_full + 13;               // [quarter]: both halves of l, l_mma written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + T::NUM_BARS);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int vh = blockIdx.x & 1;                 // value half of this CTA
+  const int unit = blockIdx.x >> 1;
+  const int row = unit / p.splits;               // b * n_q + t
+  const int split = unit % p.splits;
+  const int b = row / p.n_q;
+  const int slot_begin = split * p.slots_per_split;
+  const int slot_end = min(p.topk, slot_begin + p.slots_per_split);
+  const int n_blocks = max(0, (slot_end - slot_begin + NK - 1) / NK);
+  const int32_t* row_idx = p.indices + static_cast<size_t>(row) * p.topk;
+  const __nv_bfloat16* kv_b = p.kv + static_cast<size_t>(b) * p.n_kv * T::DQK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < T::STAGES; ++s) {
+      mbar_init(&cx_full[s], T::PRODUCERS);
+      mbar_init(&cv_full[s], T::PRODUCERS);
+      mbar_init(&cx_empty[s], 1);
+      mbar_init(&cv_empty[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, T::SOFTMAX_WARPS);
+    mbar_init(p_full, T::SOFTMAX_WARPS);
+    mbar_init(pv_done, 1);
+    mbar_init(q_ready, T::SOFTMAX_WARPS);
+    for (int s = 0; s < 12; ++s) mbar_init(&red_bar[s], 2);
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, T::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp < 4) {
+    // ------------------------------------------------------------ gather
+    // The block's 64 row indices go through a per-warp shared-memory copy
+    // (loaded one block ahead). Flat mapping: 16-byte piece c of a part
+    // (c = thread + 128 m) is piece c % per_key of key c / per_key; a thread
+    // issues all its copies back to back.
+    int32_t* sidx = reinterpret_cast<int32_t*>(smem + T::OFF_IDX) + warp * NK;
+    auto load_idx = [&](int blk, int j) -> int {
+      const int slot = slot_begin + blk * NK + j;
+      if (blk >= n_blocks || slot >= slot_end) return -1;
+      const int idx = row_idx[slot];
+      return (idx >= 0 && idx < p.n_kv) ? idx : -1;
+    };
+    auto gather_part = [&](auto per_key_c, bool vpart, uint32_t c_addr) {
+      constexpr int PER_KEY = decltype(per_key_c)::value;
+      constexpr int PER = NK * PER_KEY / T::PRODUCERS;
+#pragma unroll
+      for (int m = 0; m < PER; ++m) {
+        const int c = threadIdx.x + T::PRODUCERS * m;
+        const int j = c / PER_KEY, piece = c - j * PER_KEY;
+        const int t = piece >> 3, ch = piece & 7;
+        const int db = vpart ? 4 * vh + t : vh_xblock(t, vh);
+        const int key = sidx[j];
+        cp_async_16(c_addr + db * T::DB_BYTES + j * 128 + ((ch ^ (j & 7)) << 4),
+                    kv_b + static_cast<size_t>(key >= 0 ? key : 0) * T::DQK + db * 64 + ch * 8,
+                    key >= 0 ? 16u : 0u);
+      }
+    };
+    int next_lo = load_idx(0, lane), next_hi = load_idx(0, lane + 32);
+    bool ok = true;
+    for (int i = 0; i < n_blocks && ok; ++i) {
+      const int st = i % T::STAGES;
+      const uint32_t ph = ((i / T::STAGES) & 1) ^ 1;
+      __syncwarp();
+      sidx[lane] = next_lo;
+      sidx[lane + 32] = next_hi;
+      __syncwarp();
+      next_lo = load_idx(i + 1, lane);
+      next_hi = load_idx(i + 1, lane + 32);
+      const uint32_t c_addr = smem_u32(c_smem + st * T::STAGE_BYTES);
+      ok = mbar_wait(&cx_empty[st], ph);
+      if (!ok) break;
+      gather_part(std::integral_constant<int, T::XDB * 8>{}, false, c_addr);
+      cp_async_arrive_noinc(&cx_full[st]);
+      ok = mbar_wait(&cv_empty[st], ph);
+      if (!ok) break;
+      gather_part(std::integral_constant<int, T::VDB * 8>{}, true, c_addr);
+      cp_async_arrive_noinc(&cv_full[st]);
+    }
+    cp_async_wait_all();
+  } else if (warp == 4) {
+    // ------------------------------------------------------------ S = Q C^T issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = umma_idesc(128, NK, 1u, 1u, 0u, 0u);
+      bool ok = mbar_wait(q_ready, 0);
+      tc_fence_after();
+      for (int i = 0; i < n_blocks && ok; ++i) {
+        const int st = i % T::STAGES;
+        const uint32_t ph = (i / T::STAGES) & 1;
+        ok = mbar_wait(s_free, (i & 1) ^ 1) && mbar_wait(&cx_full[st], ph);
+        if (!ok) break;
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint32_t c_addr = smem_u32(c_smem + st * T::STAGE_BYTES);
+        // logit-only blocks, Q slice from TMEM
+#pragma unroll 1
+        for (int t = 0; t < T::XDB; ++t) {
+          const uint32_t blk = c_addr + vh_xblock(t, vh) * T::DB_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_ts(tmem_base + T::COL_S, tmem_base + T::COL_Q + t * 32 + kk * 8,
+                         umma_desc(blk + kk * 32, 16, 1024, 2), idesc_s, (t | kk) ? 1u : 0u);
+        }
+        umma_commit(&cx_empty[st]);
+        ok = mbar_wait(&cv_full[st], ph);
+        if (!ok) break;
+        fence_proxy_async_smem();
+        tc_fence_after();
+        // V-half blocks, Q slice from shared memory
+#pragma unroll 1
+        for (int u = 0; u < T::VDB; ++u) {
+          const uint32_t blk = c_addr + (4 * vh + u) * T::DB_BYTES;
+          const uint32_t qa = smem_u32(qs_smem) + u * (T::M * 128);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_ss(tmem_base + T::COL_S, umma_desc(qa + kk * 32, 16, 1024, 2),
+                         umma_desc(blk + kk * 32, 16, 1024, 2), idesc_s, 1u);
+        }
+        umma_commit(s_full);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 13) {
+    // ------------------------------------------------------------ O += P V issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_pv = umma_idesc(128, T::VH, 1u, 1u, 0u, 1u);
+      for (int j = 0; j < n_blocks; ++j) {
+        const int st = j % T::STAGES;
+        if (!mbar_wait(p_full, j & 1)) break;
+        tc_fence_after();
+        // P(j) exists only after S(j) was read, so S(j) has completed: when
+        // PV(j) completes, both readers of the V-half blocks are done.
+        const uint32_t v_addr = smem_u32(c_smem + st * T::STAGE_BYTES) + 4 * vh * T::DB_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < NK / 16; ++kk)
+          umma_bf16_ts(tmem_base + T::COL_O, tmem_base + T::COL_P + kk * 8,
+                       umma_desc(v_addr + kk * 2048, T::DB_BYTES, 1024, 2), idesc_pv,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&cv_empty[st]);
+        umma_commit(pv_done);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= 5 && warp <= 12) {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int quarter = warp & 3;
+    const int half = (warp - 5) >> 2;                        // which 32 keys of a block
+    const int h = quarter * 32 + lane;                       // head row = TMEM lane
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    float* red = reinterpret_cast<float*>(smem + T::OFF_RED);   // [parity][half][128]
+
+    // Q into TMEM (logit-only blocks; the two warps of a quarter take
+    // alternate 16-column chunks) and shared memory (V-half blocks, K-major
+    // 128-byte swizzle; each warp writes two of the four blocks).
+    {
+      const __nv_bfloat16* qh = p.q + (static_cast<size_t>(row) * p.H + min(h, p.H - 1)) * T::DQK;
+      const bool live = h < p.H;
+      for (int c = half; c < T::XDB * 2; c += 2) {
+        uint32_t v[16];
+        const uint4* src = reinterpret_cast<const uint4*>(qh + vh_xblock(c >> 1, vh) * 64 + (c & 1) * 32);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint4 u = live ? src[k] : make_uint4(0u, 0u, 0u, 0u);
+          v[4 * k] = u.x; v[4 * k + 1] = u.y; v[4 * k + 2] = u.z; v[4 * k + 3] = u.w;
+        }
+        tmem_st16(tmem_base + lane_addr + T::COL_Q + c * 16, v);
+      }
+      for (int u = 2 * half; u < 2 * half + 2; ++u) {
+        const uint4* src = reinterpret_cast<const uint4*>(qh + (4 * vh + u) * 64);
+        uint8_t* dst = qs_smem + u * (T::M * 128) + (h >> 3) * 1024 + (h & 7) * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          *reinterpret_cast<uint4*>(dst + ((ch ^ (h & 7)) << 4)) =
+              live ? src[ch] : make_uint4(0u, 0u, 0u, 0u);
+      }
+      fence_proxy_async_smem();
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+    }
+
+    float m_used = -INFINITY;   // running max (log2 domain) the P values are relative to
+    float l = 0.f;              // this warp's share of the sum of the fp32 p (LSE)
+    float l_mma = 0.f;          // ... of the bf16-rounded p the PV MMA used (normalises O)
+    bool ok = true;
+    auto load_idx = [&](int blk) -> int {
+      const int slot = slot_begin + blk * NK + half * 32 + lane;
+      return (blk < n_blocks && slot < slot_end) ? row_idx[slot] : -1;
+    };
+    int idx_next = load_idx(0);
+    uint32_t sr[32];
+    float z[32];
+    for (int i = 0; i < n_blocks && ok; ++i) {
+      // ---- logits of this warp's 32 keys; the S tile is free for S(i + 1)
+      const int idx = idx_next;
+      idx_next = load_idx(i + 1);
+      const uint32_t vmask = __ballot_sync(0xffffffffu, idx >= 0 && idx < p.n_kv);
+      if (!(ok = mbar_wait(s_full, i & 1))) break;
+      tc_fence_after();
+      tmem_ld32(tmem_base + lane_addr + T::COL_S + half * 32, sr);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+      // ---- block max over the 64 keys, shared with the partner warp
+      float hmax = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        z[j] = ((vmask >> j) & 1u) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
+        hmax = fmaxf(hmax, z[j]);
+      }
+      float* red_i = red + (i & 1) * (2 * T::M);
+      red_i[half * T::M + h] = hmax;
+      __syncwarp();
+      uint64_t* rb = &red_bar[(i & 1) * 4 + quarter];
+      if (lane == 0) mbar_arrive(rb);
+      if (!(ok = mbar_wait(rb, (i >> 1) & 1))) break;
+      const float bmax = fmaxf(hmax, red_i[(half ^ 1) * T::M + h]);
+      // ---- online softmax; P(i) into TMEM once PV(i - 1) has finished
+      const bool grow = bmax > m_used + 8.0f;
+      const float m_new = grow ? bmax : m_used;
+      if (i > 0) {
+        if (!(ok = mbar_wait(pv_done, (i - 1) & 1))) break;
+        tc_fence_after();
+      }
+      if (i > 0 && __any_sync(0xffffffffu, grow)) {
+        const float alpha = grow ? exp2f(m_used - m_new) : 1.0f;
+#pragma unroll 1
+        for (int c = half * (T::VH / 2); c < (half + 1) * (T::VH / 2); c += 16) {
+          uint32_t o[16];
+          tmem_ld16(tmem_base + lane_addr + T::COL_O + c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tmem_st16(tmem_base + lane_addr + T::COL_O + c, o);
+        }
+        tmem_wait_st();
+        l *= alpha;
+        l_mma *= alpha;
+      }
+      m_used = m_new;
+      uint32_t pk[16];
+      float lsum = 0.f, lsum_mma = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float p0 = exp2f(z[2 * j] - m_used);
+        const float p1 = exp2f(z[2 * j + 1] - m_used);
+        const __nv_bfloat162 pb2 = __floats2bfloat162_rn(p0, p1);
+        lsum += p0 + p1;
+        lsum_mma += __low2float(pb2) + __high2float(pb2);
+        pk[j] = *reinterpret_cast<const uint32_t*>(&pb2);
+      }
+      if (m_used == -INFINITY) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pk[j] = 0u;
+        lsum = 0.f;
+        lsum_mma = 0.f;
+      }
+      l += lsum;
+      l_mma += lsum_mma;
+      tmem_st16(tmem_base + lane_addr + T::COL_P + half * 16, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok && n_blocks > 0) {
+      ok = mbar_wait(pv_done, (n_blocks - 1) & 1);
+      tc_fence_after();
+    }
+    // Both warps of a quarter add their halves of l and l_mma.
+    float* red_l = reinterpret_cast<float*>(smem + T::OFF_END);   // [half][2][128]
+    red_l[(half * 2) * T::M + h] = l;
+    red_l[(half * 2 + 1) * T::M + h] = l_mma;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&end_bar[quarter]);
+    ok = mbar_wait(&end_bar[quarter], 0) && ok;
+    const float l_o = red_l[((half ^ 1) * 2) * T::M + h];
+    const float lm_o = red_l[((half ^ 1) * 2 + 1) * T::M + h];
+    const float l_all = half == 0 ? l + l_o : l_o + l;
+    const float lm_all = half == 0 ? l_mma + lm_o : lm_o + l_mma;
+    // O / sum(rounded p) is an exact convex combination of the V rows with
+    // weights perturbed by the bf16 rounding of p (a component shared by the
+    // rows cancels); the LSE keeps the unrounded sum.
+    const bool has = ok && l_all > 0.f && lm_all > 0.f;
+    const float inv_l = has ? 1.0f / lm_all : 0.f;
+    const uint32_t keep = has ? 0xffffffffu : 0u;   // masks undefined TMEM when empty
+    const float lse_v = has ? (m_used + log2f(l_all)) * 0.69314718055994531f : -INFINITY;
+    const bool direct = p.splits == 1;
+    float* dst_f32 = nullptr;
+    __nv_bfloat16* dst_bf16 = nullptr;
+    if (direct) {
+      const size_t o_off = (static_cast<size_t>(row) * p.H + h) * T::DV + vh * T::VH;
+      if (p.out_bf16) dst_bf16 = static_cast<__nv_bfloat16*>(p.out) + o_off;
+      else dst_f32 = static_cast<float*>(p.out) + o_off;
+    } else {
+      const size_t part = static_cast<size_t>(row) * p.splits + split;
+      dst_f32 = p.part_o + (part * p.H + h) * T::DV + vh * T::VH;
+    }
+#pragma unroll 1
+    for (int c = half * (T::VH / 2); c < (half + 1) * (T::VH / 2); c += 16) {
+      uint32_t o[16];
+      tmem_ld16(tmem_base + lane_addr + T::COL_O + c, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) o[j] &= keep;
+      if (h < p.H) {
+        if (dst_bf16) {
+          uint32_t pkd[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[2 * j]) * inv_l,
+                                                           __uint_as_float(o[2 * j + 1]) * inv_l);
+            pkd[j] = *reinterpret_cast<const uint32_t*>(&v);
+          }
+          reinterpret_cast<uint4*>(dst_bf16 + c)[0] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+          reinterpret_cast<uint4*>(dst_bf16 + c)[1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; j += 4)
+            reinterpret_cast<float4*>(dst_f32 + c)[j / 4] =
+                make_float4(__uint_as_float(o[j]) * inv_l, __uint_as_float(o[j + 1]) * inv_l,
+                            __uint_as_float(o[j + 2]) * inv_l, __uint_as_float(o[j + 3]) * inv_l);
+        }
+      }
+    }
+    if (vh == 0 && half == 0 && h < p.H) {
+      if (direct) {
+        if (p.lse) p.lse[static_cast<size_t>(row) * p.H + h] = lse_v;
+      } else {
+        p.part_lse[(static_cast<size_t>(row) * p.splits + split) * p.H + h] = lse_v;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, T::TMEM_COLS);
+  }
+}
+
+}  // namespace dsa
