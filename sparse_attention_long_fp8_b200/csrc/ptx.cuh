@@ -38,6 +38,18 @@ __device__ __forceinline__ uint32_t lane_id() {
   return l;
 }
 
+// True in exactly one lane of a converged warp (the lowest active lane, so
+// always the same thread when the whole warp is active). Single-thread
+// instructions (tcgen05.mma, tcgen05.commit) issued under it from warp-uniform
+// control flow keep their operands in the uniform datapath; issuing them from
+// an `if (lane == 0)` branch costs measurably more issue slots per MMA.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile("{ .reg .pred p; elect.sync _|p, 0xffffffff; selp.u32 %0, 1, 0, p; }"
+               : "=r"(pred));
+  return pred != 0;
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -50,8 +50,7 @@ struct VhTile {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int OFF_C = 0;
   static constexpr int OFF_QS = STAGES * STAGE_BYTES;
-  static constexpr int OFF_IDX = OFF_QS + QS_BYTES;          // [gather warp][NK] int32
-  static constexpr int OFF_RED = OFF_IDX + 4 * NK * 4;       // [2 parity][2 halves][128] fp32
+  static constexpr int OFF_RED = OFF_QS + QS_BYTES;          // [2 parity][2 halves][128] fp32
   static constexpr int OFF_END = OFF_RED + 2 * 2 * M * 4;    // [half][l, l_mma][128] fp32
   static constexpr int OFF_BAR = OFF_END + 2 * 2 * M * 4;
   static constexpr int NUM_BARS = 4 * STAGES + 5 + 8 + 4;    // stages, singles, red[8], end[4]
@@ -65,7 +64,7 @@ struct VhTile {
 // other half's four value blocks, then the RoPE block 8.
 __device__ __forceinline__ int vh_xblock(int t, int v) { return t == 4 ? 8 : t + 4 * (1 - v); }
 
-// Warp roles: 0-3 gather (cp.async, 16 bytes per thread and copy); 4 issues
+// Warp roles: 0-3 gather (cp.async, 16 bytes per copy); 4 issues
 // the logit MMAs and owns TMEM; 5-12 run the softmax (two warps per TMEM lane
 // quarter: a thread owns one head row and 32 of a block's 64 keys); 13 issues
 // the PV MMAs.
@@ -130,112 +129,134 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
 
   if (warp < 4) {
     // ------------------------------------------------------------ gather
-    // The block's 64 row indices go through a per-warp shared-memory copy
-    // (loaded one block ahead). Flat mapping: 16-byte piece c of a part
-    // (c = thread + 128 m) is piece c % per_key of key c / per_key; a thread
-    // issues all its copies back to back.
-    int32_t* sidx = reinterpret_cast<int32_t*>(smem + T::OFF_IDX) + warp * NK;
-    auto load_idx = [&](int blk, int j) -> int {
-      const int slot = slot_begin + blk * NK + j;
-      if (blk >= n_blocks || slot >= slot_end) return -1;
-      const int idx = row_idx[slot];
-      return (idx >= 0 && idx < p.n_kv) ? idx : -1;
-    };
-    auto gather_part = [&](auto per_key_c, bool vpart, uint32_t c_addr) {
-      constexpr int PER_KEY = decltype(per_key_c)::value;
-      constexpr int PER = NK * PER_KEY / T::PRODUCERS;
+    // Thread (kq = tid / 8, ch = tid % 8) copies 16-byte chunk ch of every
+    // 64-dim block of keys kq, kq + 16, kq + 32 and kq + 48 of a block. Under
+    // the 128-byte swizzle chunk ch of row j sits at ((ch ^ (j & 7)) << 4),
+    // and j & 7 = kq & 7 for all four keys: the shared-memory destination is
+    // a per-thread constant plus an immediate and the source a row pointer
+    // plus an immediate, so a copy costs about one issued instruction. A warp
+    // instruction moves four whole 128-byte lines.
+    const int kq = threadIdx.x >> 3, ch = threadIdx.x & 7;
+    const uint32_t dst0 = smem_u32(c_smem) + kq * 128 + ((ch ^ (kq & 7)) << 4);
+    auto load_keys = [&](int blk, int (&k)[4]) {
 #pragma unroll
-      for (int m = 0; m < PER; ++m) {
-        const int c = threadIdx.x + T::PRODUCERS * m;
-        const int j = c / PER_KEY, piece = c - j * PER_KEY;
-        const int t = piece >> 3, ch = piece & 7;
-        const int db = vpart ? 4 * vh + t : vh_xblock(t, vh);
-        const int key = sidx[j];
-        cp_async_16(c_addr + db * T::DB_BYTES + j * 128 + ((ch ^ (j & 7)) << 4),
-                    kv_b + static_cast<size_t>(key >= 0 ? key : 0) * T::DQK + db * 64 + ch * 8,
-                    key >= 0 ? 16u : 0u);
+      for (int r = 0; r < 4; ++r) {
+        const int slot = slot_begin + blk * NK + kq + 16 * r;
+        const int idx = (blk < n_blocks && slot < slot_end) ? row_idx[slot] : -1;
+        k[r] = (idx >= 0 && idx < p.n_kv) ? idx : -1;
       }
     };
-    int next_lo = load_idx(0, lane), next_hi = load_idx(0, lane + 32);
+    auto copy_part = [&](auto vh_c, auto vpart_c, uint32_t dst, const __nv_bfloat16* const (&src)[4],
+                         const uint32_t (&bytes)[4]) {
+      constexpr int V = decltype(vh_c)::value;
+      constexpr bool VP = decltype(vpart_c)::value;
+#pragma unroll
+      for (int t = 0; t < (VP ? T::VDB : T::XDB); ++t) {
+        const int db = VP ? 4 * V + t : (t == 4 ? 8 : t + 4 * (1 - V));
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          cp_async_16(dst + db * T::DB_BYTES + r * 16 * 128, src[r] + db * 64, bytes[r]);
+      }
+    };
+    using I0 = std::integral_constant<int, 0>;
+    using I1 = std::integral_constant<int, 1>;
+    using BX = std::integral_constant<bool, false>;
+    using BV = std::integral_constant<bool, true>;
+    int keys[4];
+    load_keys(0, keys);
     bool ok = true;
     for (int i = 0; i < n_blocks && ok; ++i) {
       const int st = i % T::STAGES;
       const uint32_t ph = ((i / T::STAGES) & 1) ^ 1;
-      __syncwarp();
-      sidx[lane] = next_lo;
-      sidx[lane + 32] = next_hi;
-      __syncwarp();
-      next_lo = load_idx(i + 1, lane);
-      next_hi = load_idx(i + 1, lane + 32);
-      const uint32_t c_addr = smem_u32(c_smem + st * T::STAGE_BYTES);
+      const __nv_bfloat16* src[4];
+      uint32_t bytes[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        src[r] = kv_b + static_cast<size_t>(keys[r] >= 0 ? keys[r] : 0) * T::DQK + ch * 8;
+        bytes[r] = keys[r] >= 0 ? 16u : 0u;
+      }
+      load_keys(i + 1, keys);   // one block ahead
+      const uint32_t dst = dst0 + st * T::STAGE_BYTES;
       ok = mbar_wait(&cx_empty[st], ph);
       if (!ok) break;
-      gather_part(std::integral_constant<int, T::XDB * 8>{}, false, c_addr);
+      if (vh == 0) copy_part(I0{}, BX{}, dst, src, bytes);
+      else copy_part(I1{}, BX{}, dst, src, bytes);
       cp_async_arrive_noinc(&cx_full[st]);
       ok = mbar_wait(&cv_empty[st], ph);
       if (!ok) break;
-      gather_part(std::integral_constant<int, T::VDB * 8>{}, true, c_addr);
+      if (vh == 0) copy_part(I0{}, BV{}, dst, src, bytes);
+      else copy_part(I1{}, BV{}, dst, src, bytes);
       cp_async_arrive_noinc(&cv_full[st]);
     }
     cp_async_wait_all();
   } else if (warp == 4) {
     // ------------------------------------------------------------ S = Q C^T issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = umma_idesc(128, NK, 1u, 1u, 0u, 0u);
-      bool ok = mbar_wait(q_ready, 0);
+    // The whole warp runs the loop; one elected lane issues. Descriptors are
+    // formed once: adding (byte offset >> 4) to a descriptor moves its start
+    // address (every shared address here is below 256 KB, so the 14-bit
+    // field cannot carry).
+    constexpr uint32_t idesc_s = umma_idesc(128, NK, 1u, 1u, 0u, 0u);
+    const uint64_t c_desc0 = umma_desc(smem_u32(c_smem), 16, 1024, 2);
+    const uint64_t q_desc0 = umma_desc(smem_u32(qs_smem), 16, 1024, 2);
+    const uint32_t x_shift = static_cast<uint32_t>(4 * (1 - vh) * T::DB_BYTES) >> 4;
+    const uint32_t v_shift = static_cast<uint32_t>(4 * vh * T::DB_BYTES) >> 4;
+    bool ok = mbar_wait(q_ready, 0);
+    tc_fence_after();
+    for (int i = 0; i < n_blocks && ok; ++i) {
+      const int st = i % T::STAGES;
+      const uint32_t ph = (i / T::STAGES) & 1;
+      ok = mbar_wait(s_free, (i & 1) ^ 1) && mbar_wait(&cx_full[st], ph);
+      if (!ok) break;
+      fence_proxy_async_smem();
       tc_fence_after();
-      for (int i = 0; i < n_blocks && ok; ++i) {
-        const int st = i % T::STAGES;
-        const uint32_t ph = (i / T::STAGES) & 1;
-        ok = mbar_wait(s_free, (i & 1) ^ 1) && mbar_wait(&cx_full[st], ph);
-        if (!ok) break;
-        fence_proxy_async_smem();
-        tc_fence_after();
-        const uint32_t c_addr = smem_u32(c_smem + st * T::STAGE_BYTES);
-        // logit-only blocks, Q slice from TMEM
-#pragma unroll 1
-        for (int t = 0; t < T::XDB; ++t) {
-          const uint32_t blk = c_addr + vh_xblock(t, vh) * T::DB_BYTES;
+      const uint64_t cd = c_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
+      // logit-only blocks (the other half's value blocks, then RoPE block 8),
+      // Q slice from TMEM
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_ts(tmem_base + T::COL_S, tmem_base + T::COL_Q + t * 32 + kk * 8,
-                         umma_desc(blk + kk * 32, 16, 1024, 2), idesc_s, (t | kk) ? 1u : 0u);
-        }
-        umma_commit(&cx_empty[st]);
-        ok = mbar_wait(&cv_full[st], ph);
-        if (!ok) break;
-        fence_proxy_async_smem();
-        tc_fence_after();
-        // V-half blocks, Q slice from shared memory
-#pragma unroll 1
-        for (int u = 0; u < T::VDB; ++u) {
-          const uint32_t blk = c_addr + (4 * vh + u) * T::DB_BYTES;
-          const uint32_t qa = smem_u32(qs_smem) + u * (T::M * 128);
+      for (int t = 0; t < T::XDB; ++t)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_ss(tmem_base + T::COL_S, umma_desc(qa + kk * 32, 16, 1024, 2),
-                         umma_desc(blk + kk * 32, 16, 1024, 2), idesc_s, 1u);
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bd = t < 4 ? cd + x_shift + ((t * T::DB_BYTES + kk * 32) >> 4)
+                                    : cd + ((8 * T::DB_BYTES + kk * 32) >> 4);
+          if (elect_one())
+            umma_bf16_ts(tmem_base + T::COL_S, tmem_base + T::COL_Q + t * 32 + kk * 8, bd,
+                         idesc_s, (t | kk) ? 1u : 0u);
         }
-        umma_commit(s_full);
-      }
+      if (elect_one()) umma_commit(&cx_empty[st]);
+      ok = mbar_wait(&cv_full[st], ph);
+      if (!ok) break;
+      fence_proxy_async_smem();
+      tc_fence_after();
+      // V-half blocks, Q slice from shared memory
+#pragma unroll
+      for (int u = 0; u < T::VDB; ++u)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = q_desc0 + ((u * T::M * 128 + kk * 32) >> 4);
+          const uint64_t bd = cd + v_shift + ((u * T::DB_BYTES + kk * 32) >> 4);
+          if (elect_one()) umma_bf16_ss(tmem_base + T::COL_S, ad, bd, idesc_s, 1u);
+        }
+      if (elect_one()) umma_commit(s_full);
     }
     __syncwarp();
   } else if (warp == 13) {
     // ------------------------------------------------------------ O += P V issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_pv = umma_idesc(128, T::VH, 1u, 1u, 0u, 1u);
-      for (int j = 0; j < n_blocks; ++j) {
-        const int st = j % T::STAGES;
-        if (!mbar_wait(p_full, j & 1)) break;
-        tc_fence_after();
-        // P(j) exists only after S(j) was read, so S(j) has completed: when
-        // PV(j) completes, both readers of the V-half blocks are done.
-        const uint32_t v_addr = smem_u32(c_smem + st * T::STAGE_BYTES) + 4 * vh * T::DB_BYTES;
+    constexpr uint32_t idesc_pv = umma_idesc(128, T::VH, 1u, 1u, 0u, 1u);
+    const uint64_t v_desc0 =
+        umma_desc(smem_u32(c_smem) + 4 * vh * T::DB_BYTES, T::DB_BYTES, 1024, 2);
+    for (int j = 0; j < n_blocks; ++j) {
+      const int st = j % T::STAGES;
+      if (!mbar_wait(p_full, j & 1)) break;
+      tc_fence_after();
+      // P(j) exists only after S(j) was read, so S(j) has completed: when
+      // PV(j) completes, both readers of the V-half blocks are done.
+      const uint64_t vd = v_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
 #pragma unroll
-        for (int kk = 0; kk < NK / 16; ++kk)
+      for (int kk = 0; kk < NK / 16; ++kk)
+        if (elect_one())
           umma_bf16_ts(tmem_base + T::COL_O, tmem_base + T::COL_P + kk * 8,
-                       umma_desc(v_addr + kk * 2048, T::DB_BYTES, 1024, 2), idesc_pv,
-                       (j > 0 || kk > 0) ? 1u : 0u);
+                       vd + ((kk * 2048) >> 4), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+      if (elect_one()) {
         umma_commit(&cv_empty[st]);
         umma_commit(pv_done);
       }
