@@ -4,10 +4,11 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 A step is one pass of the whole path over one batch of synthetic input: the
-lightning indexer and top-k over every row chunk, then the sparse attention
-over all rows, composed from the library's stage calls exactly as
-dsa_forward launches them, so each kernel can be timed with CUDA events on
-its stream. The headline workload is DSA prefill at L = 65536 (batch 1,
+lightning indexer with its top-k selection (one fused kernel for prefill; a
+score kernel and a selection kernel per row chunk for decode), then the
+sparse attention over all rows, composed from the library's stage calls
+exactly as dsa_forward launches them, so each kernel can be timed with CUDA
+events on its stream. The headline workload is DSA prefill at L = 65536 (batch 1,
 H^I = 64, d^I = 128, k = 2048, 128-head MQA over the 576-d latent); batch
 decode (64 x 32768 and 64 x 65536 cached tokens) is measured after it.
 
@@ -174,7 +175,6 @@ class Step:
         self.chunk = dsa.forward_chunk_rows(self.shape)
         self.attn_ws_bytes = dsa.workspace_size(self.shape, dsa.DSA_OP_SPARSE_ATTN)
         self.fwd_ws_bytes = dsa.workspace_size(self.shape, dsa.DSA_OP_FORWARD)
-        self.scores = torch.empty(B, min(self.chunk, T), cfg.n_kv, device=device)
         self.attn_ws = torch.empty(max(self.attn_ws_bytes, 256), dtype=torch.uint8, device=device)
         self.idx = torch.empty(B, T, cfg.topk, dtype=torch.int32, device=device)
         self.out = torch.empty(B, T, cfg.heads, cfg.v_dim, device=device)
@@ -182,7 +182,13 @@ class Step:
         self.chunks = [(r0, min(T, r0 + self.chunk)) for r0 in range(0, T, self.chunk)]
         if B > 1 and len(self.chunks) > 1:
             raise ValueError("stage composition needs one chunk when batch > 1")
-        self.launches = 2 * len(self.chunks) + 1 + (1 if self.attn_ws_bytes > 0 else 0)
+        # dsa_forward's plan: the fused indexer + selection needs no score
+        # buffer, so its forward workspace is the attention's alone.
+        self.fused = self.fwd_ws_bytes == self.attn_ws_bytes
+        self.scores = None if self.fused else torch.empty(B, min(self.chunk, T), cfg.n_kv,
+                                                          device=device)
+        per_chunk = 1 if self.fused else 2
+        self.launches = per_chunk * len(self.chunks) + 1 + (1 if self.attn_ws_bytes > 0 else 0)
 
     def run(self, ev=None):
         """One step; with ev = (list of (start, end) event pairs per stage) the
@@ -190,7 +196,12 @@ class Step:
         dsa, x, cfg = self.dsa, self.inp, self.cfg
         rec = (lambda name: ev[name].append(self.torch.cuda.Event(enable_timing=True)) or
                ev[name][-1].record()) if ev is not None else (lambda name: None)
-        for r0, r1 in self.chunks:
+        if self.fused:
+            rec("indexer")
+            dsa.dsa_indexer_topk(self.shape, x["q_fp8"], x["q_scale"], x["w"], x["k_fp8"],
+                                 x["k_scale"], x["q_pos0"], x["kv_len"], 0, cfg.n_q, self.idx)
+            rec("indexer")
+        for r0, r1 in ([] if self.fused else self.chunks):
             rec("indexer")
             dsa.dsa_indexer_scores(self.shape, x["q_fp8"], x["q_scale"], x["w"], x["k_fp8"],
                                    x["k_scale"], x["q_pos0"], x["kv_len"], r0, r1, self.scores,
@@ -388,6 +399,7 @@ def main():
     clocks.start()
     ms, stages = timed(step, args.steps, args.warmup, dist)
     clock_info = clocks.stop()
+    fused = step.fused
     del step
     torch.cuda.empty_cache()
 
@@ -401,12 +413,13 @@ def main():
     ix_tf = ix_f / (ix_ms / 1e3) / 1e12
     at_tf = at_f / (at_ms / 1e3) / 1e12
     dominant = max(("indexer", ix_ms), ("attn", at_ms), ("topk", tk_ms), key=lambda x: x[1])[0]
+    ix_kernel = "indexer_topk_kernel<64,128,4>" if fused else "indexer_scores_kernel<64,128,4>"
     if dominant == "attn":
-        roof = {"kernel": "sparse_attn_kernel<576,512,2>", "bound": "tensor",
+        roof = {"kernel": "sparse_attn_vh_kernel", "bound": "tensor",
                 "achieved": at_f / (at_ms / 1e3) / 1e12, "peak": peaks["bf16_sustained"],
                 "unit": "TFLOP/s", "traffic": None}
     elif dominant == "indexer":
-        roof = {"kernel": "indexer_scores_kernel<64,128,4>", "bound": "tensor",
+        roof = {"kernel": ix_kernel, "bound": "tensor",
                 "achieved": ix_tf, "peak": fp8_peak, "unit": "TFLOP/s", "traffic": None}
     else:
         roof = {"kernel": "topk_kernel", "bound": "hbm", "achieved": None,
@@ -427,7 +440,8 @@ def main():
                    "heads": cfg.heads, "qk_dim": cfg.qk_dim, "v_dim": cfg.v_dim,
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (q is 9.7 GB per step)"},
-        "stages_ms": {"indexer": ix_ms, "topk": tk_ms, "attention": at_ms},
+        "stages_ms": ({"indexer_topk_fused": ix_ms, "attention": at_ms} if fused else
+                      {"indexer": ix_ms, "topk": tk_ms, "attention": at_ms}),
         "indexer_tflops_fp8": ix_tf, "indexer_frac_fp8": ix_tf / fp8_peak,
         "attention_tflops_bf16": at_tf, "attention_frac_bf16": at_tf / peaks["bf16_sustained"],
         "roofline": roof, "gpu_launches": step_launches_total(stages),

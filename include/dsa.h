@@ -101,6 +101,29 @@ dsa_status dsa_indexer_scores(const dsa_shape* shape, const uint8_t* q_fp8,
                               int32_t flags, float* scores, void* stream);
 
 /*
+ * Indexer scores and top-k selection in one kernel (page "DeepseekV3.2 拆解",
+ * section "闪电索引器", eq. I_{t,s}, and section "细粒度 Token 选择机制",
+ * eq. u_t). Inputs and row range as dsa_indexer_scores; the score of each
+ * (row, key) pair is computed exactly as dsa_indexer_scores computes it but
+ * is never written to memory: each row keeps its candidates in shared memory
+ * and only the selection leaves the GPU's SMs.
+ *   indices [B, row_end-row_begin, topk] int32, as dsa_topk writes them:
+ *           min(m, topk) distinct key indices of the m visible keys (the
+ *           largest scores, ties to the lower index), then -1 padding, in
+ *           unspecified order within a row.
+ *   Supported: idx_heads = 64, idx_dim = 128, topk <= 2048; otherwise
+ *   DSA_ERR_UNSUPPORTED before any launch (use dsa_indexer_scores + dsa_topk).
+ *   No workspace. dsa_forward uses this kernel whenever the shape is
+ *   supported and there are at least as many 4-row query groups as SMs.
+ */
+dsa_status dsa_indexer_topk(const dsa_shape* shape, const uint8_t* q_fp8,
+                            const float* q_scale, const float* w,
+                            const uint8_t* k_fp8, const float* k_scale,
+                            const int32_t* q_pos0, const int32_t* kv_len,
+                            int32_t row_begin, int32_t row_end, int32_t* indices,
+                            void* stream);
+
+/*
  * Top-k selection per score row (page "DeepseekV3.2 拆解", eq. u_t: keep the
  * k keys with the largest I[t,s]).
  *   scores  [B, row_end-row_begin, n_kv] fp32 (as written by

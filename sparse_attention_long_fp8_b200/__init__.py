@@ -70,6 +70,7 @@ def load_library(path: str | None = None):
     P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     SP = ctypes.POINTER(DsaShape)
     lib.dsa_indexer_scores.argtypes = [SP, P, P, P, P, P, P, P, I32, I32, I32, P, P]
+    lib.dsa_indexer_topk.argtypes = [SP, P, P, P, P, P, P, P, I32, I32, P, P]
     lib.dsa_topk.argtypes = [SP, P, I32, I32, P, P, P, P, SZ, P]
     lib.dsa_sparse_attn.argtypes = [SP, P, P, P, P, I32, P, P, SZ, P]
     lib.dsa_sparse_attn_noalloc.argtypes = [SP, P, P, P, P, I32, P, P]
@@ -81,7 +82,7 @@ def load_library(path: str | None = None):
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_last_error.restype = ctypes.c_char_p
     lib.dsa_version.restype = ctypes.c_char_p
-    for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
+    for fn in ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
                "dsa_workspace_size", "dsa_check", "dsa_forward_chunk_rows",
                "dsa_sparse_attn_noalloc"):
         getattr(lib, fn).restype = ctypes.c_int
@@ -153,6 +154,16 @@ def dsa_indexer_scores(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
         _ptr(q_pos0, d["i32"], "q_pos0"), _ptr(kv_len, d["i32"], "kv_len"),
         int(row_begin), int(row_end), int(flags), _ptr(scores, d["f32"], "scores"),
         _stream(stream)))
+
+
+def dsa_indexer_topk(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+                     row_begin, row_end, indices, stream=None):
+    d = _dt()
+    _raise(load_library().dsa_indexer_topk(
+        ctypes.byref(shape), _ptr(q_fp8, d["u8"], "q_fp8"), _ptr(q_scale, d["f32"], "q_scale"),
+        _ptr(w, d["f32"], "w"), _ptr(k_fp8, d["u8"], "k_fp8"), _ptr(k_scale, d["f32"], "k_scale"),
+        _ptr(q_pos0, d["i32"], "q_pos0"), _ptr(kv_len, d["i32"], "kv_len"),
+        int(row_begin), int(row_end), _ptr(indices, d["i32"], "indices"), _stream(stream)))
 
 
 def dsa_topk(shape, scores, row_begin, row_end, q_pos0, kv_len, indices, ws=None,

@@ -15,6 +15,7 @@
 
 #include "../../include/dsa.h"
 #include "indexer.cuh"
+#include "indexer_topk.cuh"
 #include "sparse_attn.cuh"
 #include "sparse_attn_vh.cuh"
 #include "topk.cuh"
@@ -231,6 +232,49 @@ dsa_status launch_indexer(const dsa_shape* s, const uint8_t* q_fp8, const float*
                                      row_begin, rows, scores, write_invalid, stream, dev);
 }
 
+// Scores and selection in one kernel: H^I = 64, d^I = 128, k <= 2048.
+bool indexer_topk_supported(const dsa_shape* s) {
+  using T = dsa::IndexerTopkTile<64, 128, 4>;
+  return s->idx_heads == 64 && s->idx_dim == 128 && s->topk <= T::MAX_K;
+}
+
+dsa_status launch_indexer_topk(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
+                               const float* w, const uint8_t* k_fp8, const float* k_scale,
+                               const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
+                               int32_t rows, int32_t* indices, int32_t out_rows,
+                               cudaStream_t stream, int dev) {
+  using T = dsa::IndexerTopkTile<64, 128, 4>;
+  static bool attr_done[kMaxDevices] = {false};
+  if (dsa_status st = set_smem(dsa::indexer_topk_kernel<64, 128, 4>, T::SMEM_BYTES, dev, attr_done))
+    return st;
+  if (rows <= 0) return DSA_OK;
+  CUtensorMap tq, tk;
+  if (dsa_status st = make_tmap_u8(&tq, q_fp8, static_cast<uint64_t>(s->batch) * s->n_q * 64, 128, T::N))
+    return st;
+  if (dsa_status st = make_tmap_u8(&tk, k_fp8, static_cast<uint64_t>(s->batch) * s->n_kv, 128, T::M))
+    return st;
+  dsa::IndexerTopkParams p{};
+  p.q_scale = q_scale;
+  p.w = w;
+  p.k_scale = k_scale;
+  p.q_pos0 = q_pos0;
+  p.kv_len = kv_len;
+  p.indices = indices;
+  p.B = s->batch;
+  p.n_q = s->n_q;
+  p.n_kv = s->n_kv;
+  p.k = s->topk;
+  p.row_begin = row_begin;
+  p.rows = rows;
+  p.n_groups = (rows + 3) / 4;
+  p.out_rows = out_rows;
+  if (s->batch > 65535) return fail(DSA_ERR_INVALID_ARG, "batch > 65535");
+  dim3 grid(p.n_groups, s->batch);
+  dsa::indexer_topk_kernel<64, 128, 4><<<grid, T::THREADS, T::SMEM_BYTES, stream>>>(tq, tk, p);
+  DSA_CUDA_TRY(cudaGetLastError(), "fused indexer top-k launch");
+  return DSA_OK;
+}
+
 // ------------------------------------------------------------------ top-k launch
 
 dsa_status launch_topk(const dsa_shape* s, const float* scores, int32_t row_begin, int32_t rows,
@@ -393,11 +437,24 @@ dsa_status launch_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv
 
 struct FwdPlan {
   int chunk_rows;
+  bool fused;   // scores and selection in one kernel: no score buffer at all
   size_t scores_bytes, attn_bytes, total;
 };
 
 FwdPlan plan_forward(const dsa_shape* s) {
   FwdPlan f{};
+  f.attn_bytes = plan_attn(s).ws_bytes;
+  // The fused kernel runs one CTA per 4 query rows over all of their keys;
+  // with fewer groups than SMs (decode) the split score kernel plus the
+  // separate selection keeps more of the GPU busy.
+  const int64_t groups = static_cast<int64_t>(s->batch) * ((s->n_q + 3) / 4);
+  if (indexer_topk_supported(s) && groups >= kNumSms) {
+    f.fused = true;
+    f.chunk_rows = s->n_q;
+    f.scores_bytes = 0;
+    f.total = f.attn_bytes;
+    return f;
+  }
   const size_t row_bytes = static_cast<size_t>(s->batch) * s->n_kv * sizeof(float);
   const size_t budget = 256ull << 20;   // scores of one row chunk (L2-sized pieces at 64K+)
   int64_t chunk = static_cast<int64_t>(budget / row_bytes);
@@ -406,7 +463,6 @@ FwdPlan plan_forward(const dsa_shape* s) {
   if (chunk < s->n_q) chunk = std::max<int64_t>(64, chunk / 64 * 64);
   f.chunk_rows = static_cast<int>(chunk);
   f.scores_bytes = (row_bytes * chunk + 255) / 256 * 256;
-  f.attn_bytes = plan_attn(s).ws_bytes;
   f.total = f.scores_bytes + f.attn_bytes;
   return f;
 }
@@ -519,6 +575,31 @@ dsa_status dsa_indexer_scores(const dsa_shape* s, const uint8_t* q_fp8, const fl
                         static_cast<cudaStream_t>(stream), dev);
 }
 
+dsa_status dsa_indexer_topk(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
+                            const float* w, const uint8_t* k_fp8, const float* k_scale,
+                            const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
+                            int32_t row_end, int32_t* indices, void* stream) {
+  if (dsa_status st = check_indexer_shape(s)) return st;
+  if (dsa_status st = check_topk_shape(s)) return st;
+  if (!indexer_topk_supported(s))
+    return fail(DSA_ERR_UNSUPPORTED,
+                "dsa_indexer_topk supports idx_heads = 64, idx_dim = 128, topk <= 2048 "
+                "(got %d, %d, %d)",
+                s->idx_heads, s->idx_dim, s->topk);
+  if (dsa_status st = check_ptrs({q_fp8, q_scale, w, k_fp8, k_scale, indices}, "dsa_indexer_topk"))
+    return st;
+  if (row_begin < 0 || row_end > s->n_q || row_begin >= row_end)
+    return fail(DSA_ERR_INVALID_ARG, "row range [%d, %d) outside [0, %d) or empty", row_begin,
+                row_end, s->n_q);
+  if (!aligned(q_fp8, 16) || !aligned(k_fp8, 16))
+    return fail(DSA_ERR_INVALID_ARG, "q_fp8 and k_fp8 must be 16-byte aligned");
+  int dev;
+  if (dsa_status st = current_device(&dev)) return st;
+  return launch_indexer_topk(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, row_begin,
+                             row_end - row_begin, indices, row_end - row_begin,
+                             static_cast<cudaStream_t>(stream), dev);
+}
+
 dsa_status dsa_topk(const dsa_shape* s, const float* scores, int32_t row_begin, int32_t row_end,
                     const int32_t* q_pos0, const int32_t* kv_len, int32_t* indices, void* ws,
                     size_t ws_bytes, void* stream) {
@@ -592,15 +673,24 @@ dsa_status dsa_forward(const dsa_shape* s, const uint8_t* q_fp8, const float* q_
       !aligned(out, 16))
     return fail(DSA_ERR_INVALID_ARG, "q_fp8, k_fp8, q, kv and out must be 16-byte aligned");
   const FwdPlan f = plan_forward(s);
-  if (!ws || ws_bytes < f.total)
-    return fail(DSA_ERR_WORKSPACE, "dsa_forward needs %zu workspace bytes, got %zu", f.total,
-                ws ? ws_bytes : size_t(0));
-  if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (f.total > 0) {
+    if (!ws || ws_bytes < f.total)
+      return fail(DSA_ERR_WORKSPACE, "dsa_forward needs %zu workspace bytes, got %zu", f.total,
+                  ws ? ws_bytes : size_t(0));
+    if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  }
   int dev;
   if (dsa_status st = current_device(&dev)) return st;
   cudaStream_t st_ = static_cast<cudaStream_t>(stream);
   float* scores = static_cast<float*>(ws);
   void* attn_ws = static_cast<char*>(ws) + f.scores_bytes;
+  if (f.fused) {
+    if (dsa_status e = launch_indexer_topk(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+                                           0, s->n_q, indices_out, s->n_q, st_, dev))
+      return e;
+    return launch_attn(s, q, kv, indices_out, out, out_dtype == DSA_OUT_BF16, lse, attn_ws,
+                       f.attn_bytes, st_, dev);
+  }
   for (int r0 = 0; r0 < s->n_q; r0 += f.chunk_rows) {
     const int rows = std::min(f.chunk_rows, s->n_q - r0);
     if (dsa_status e = launch_indexer(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, r0,
@@ -626,6 +716,8 @@ dsa_status dsa_check(void* stream) {
     cudaMemcpyToSymbol(dsa::g_error_word, &zero, sizeof(zero));
     if (word & dsa::kErrTimeout)
       return fail(DSA_ERR_TIMEOUT, "a device-side wait exceeded its limit (error word 0x%x)", word);
+    if (word & dsa::kErrInternal)
+      return fail(DSA_ERR_CUDA, "a kernel invariant failed (error word 0x%x)", word);
     return fail(DSA_ERR_CUDA, "device error word 0x%x", word);
   }
   return DSA_OK;

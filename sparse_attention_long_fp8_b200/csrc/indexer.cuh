@@ -71,8 +71,7 @@ __global__ void __launch_bounds__(IndexerTile<HI, DI, QG>::THREADS, 1)
                           const __grid_constant__ CUtensorMap tmap_k, IndexerParams p) {
   using T = IndexerTile<HI, DI, QG>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   uint8_t* q_smem = smem + T::OFF_Q;
   uint8_t* k_smem = smem + T::OFF_K;
   float* coef = reinterpret_cast<float*>(smem + T::OFF_COEF);

@@ -15,11 +15,38 @@ namespace dsa {
 __device__ unsigned int g_error_word;
 
 constexpr unsigned int kErrTimeout = 1u;
+// A kernel found one of its own invariants broken (a bug, never an input error).
+constexpr unsigned int kErrInternal = 2u;
 // Bounded waits give up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Explicit shared-memory loads by 32-bit shared-window address (for data
+// reached through pointers whose address space the compiler cannot see).
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// The first 1024-byte aligned byte of a dynamic shared-memory array. The
+// offset is computed from the shared-window address and applied to the array
+// pointer itself, so the compiler still knows the result points to shared
+// memory and emits shared-memory loads, stores and atomics through it (a
+// round trip through an integer would make them generic).
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* smem_raw) {
+  return smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 }
 
 __device__ __forceinline__ unsigned long long globaltimer() {

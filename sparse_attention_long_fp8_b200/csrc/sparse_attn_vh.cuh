@@ -72,8 +72,7 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
   using T = VhTile;
   constexpr int NK = T::NK;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   uint8_t* c_smem = smem + T::OFF_C;
   uint8_t* qs_smem = smem + T::OFF_QS;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::OFF_BAR);

@@ -28,7 +28,7 @@ def _declared_functions():
 
 def test_header_declares_the_path_calls():
     names = _declared_functions()
-    for n in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
+    for n in ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
               "dsa_workspace_size", "dsa_check", "dsa_status_string", "dsa_last_error"):
         assert n in names
 
@@ -51,6 +51,21 @@ def _call_indexer(lib, shape, rb=0, re_=16, ptrs=None, flags=0):
     return lib.dsa_indexer_scores(ctypes.byref(shape) if shape is not None else None,
                                   p[0], p[1], p[2], p[3], p[4], None, None, rb, re_, flags,
                                   FAKE, None)
+
+
+def test_indexer_topk_rejects_unsupported_shapes_before_launch(lib):
+    tiny = dsa.shape_of(dsa.CONFIGS["tiny"])
+    st = lib.dsa_indexer_topk(ctypes.byref(tiny), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 0, 16,
+                              FAKE, None)
+    assert st == dsa.DSA_ERR_UNSUPPORTED
+    big_k = _shape(topk=4096)
+    st = lib.dsa_indexer_topk(ctypes.byref(big_k), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 0, 16,
+                              FAKE, None)
+    assert st == dsa.DSA_ERR_UNSUPPORTED
+    ok_shape = _shape()
+    st = lib.dsa_indexer_topk(ctypes.byref(ok_shape), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 5, 5,
+                              FAKE, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG
 
 
 def test_status_strings(lib):
@@ -108,19 +123,28 @@ def test_bad_out_dtype_and_workspace(lib):
     shape = _shape()
     assert lib.dsa_sparse_attn(ctypes.byref(shape), FAKE, FAKE, FAKE, FAKE, 7, None, None, 0,
                                None) == dsa.DSA_ERR_INVALID_ARG
-    st = lib.dsa_forward(ctypes.byref(shape), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE,
+    dec = dsa.shape_of(dsa.CONFIGS["decode_32k"])   # the two-pass plan needs a score buffer
+    st = lib.dsa_forward(ctypes.byref(dec), FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE,
                          FAKE, FAKE, FAKE, 0, None, None, 0, None)
     assert st == dsa.DSA_ERR_WORKSPACE
 
 
 def test_workspace_sizes(lib):
-    # prefill at 4K: one score chunk of 4096 x 4096 fp32, no split-K partials
-    assert dsa.workspace_size(_shape(), dsa.DSA_OP_FORWARD) == 4096 * 4096 * 4
+    # prefill: scores and selection are fused, so no score buffer and no
+    # split-K partials
+    assert dsa.workspace_size(_shape(), dsa.DSA_OP_FORWARD) == 0
     assert dsa.workspace_size(_shape(), dsa.DSA_OP_SPARSE_ATTN) == 0
     assert dsa.workspace_size(_shape(), dsa.DSA_OP_TOPK) == 0
-    # 64K: scores are chunked (256 MB of rows at a time), never the full L x L
     big = dsa.shape_of(dsa.CONFIGS["prefill_64k"])
-    assert dsa.workspace_size(big, dsa.DSA_OP_FORWARD) == 1024 * 65536 * 4
+    assert dsa.workspace_size(big, dsa.DSA_OP_FORWARD) == 0
+    assert dsa.forward_chunk_rows(big) == 65536
+    # decode (64 query groups < SMs): the split score kernel writes one chunk
+    # of 64 x 32768 fp32 scores, then the separate selection runs
+    dec = dsa.shape_of(dsa.CONFIGS["decode_32k"])
+    assert dsa.workspace_size(dec, dsa.DSA_OP_FORWARD) >= 64 * 32768 * 4
+    # the tiny shape is not supported by the fused kernel: two passes
+    tiny = dsa.shape_of(dsa.CONFIGS["tiny"])
+    assert dsa.workspace_size(tiny, dsa.DSA_OP_FORWARD) == 256 * 256 * 4
     # a handful of rows: split-K partials are needed
     few = _shape(n_q=4)
     assert dsa.workspace_size(few, dsa.DSA_OP_SPARSE_ATTN) > 0

@@ -141,6 +141,83 @@ def test_topk_band_on_gpu_scores_4k():
     check_topk_band(got[SAMPLE_4K], _oracle_scores(cfg, inp, 0, SAMPLE_4K), cfg.topk)
 
 
+# ------------------------------------------------------------------ fused indexer + top-k
+
+def _two_pass(cfg, g, rb, re_):
+    sc = _gpu_scores(cfg, g, rb, re_)
+    idx = torch.empty(cfg.batch, re_ - rb, cfg.topk, dtype=torch.int32, device="cuda")
+    dsa.dsa_topk(dsa.shape_of(cfg), sc, rb, re_, g["q_pos0"], g["kv_len"], idx)
+    dsa.dsa_check()
+    return idx
+
+
+def _fused(cfg, g, rb, re_):
+    idx = torch.full((cfg.batch, re_ - rb, cfg.topk), -7, dtype=torch.int32, device="cuda")
+    dsa.dsa_indexer_topk(dsa.shape_of(cfg), g["q_fp8"], g["q_scale"], g["w"], g["k_fp8"],
+                         g["k_scale"], g["q_pos0"], g["kv_len"], rb, re_, idx)
+    dsa.dsa_check()
+    return idx
+
+
+def _assert_same_sets(a, b):
+    """Both kernels form each score with the same fp32 operations, so the
+    selected sets must be identical (integer work: bit-exact)."""
+    a = np.sort(a.cpu().numpy(), axis=-1)
+    b = np.sort(b.cpu().numpy(), axis=-1)
+    bad = np.nonzero((a != b).any(axis=-1))
+    assert a.shape == b.shape and len(bad[0]) == 0, f"rows differ: {list(zip(*bad))[:8]}"
+
+
+def test_indexer_topk_equals_two_pass_4k():
+    cfg, inp, g = _inputs("prefill_4k")
+    fused = _fused(cfg, g, 0, cfg.n_q)
+    _assert_same_sets(fused, _two_pass(cfg, g, 0, cfg.n_q))
+    check_topk_band(fused.cpu().numpy()[0][SAMPLE_4K], _oracle_scores(cfg, inp, 0, SAMPLE_4K),
+                    cfg.topk)
+
+
+@pytest.mark.parametrize("n,kvl,pos0,rb,re_", [(300, 300, 0, 0, 300), (301, 257, 0, 3, 298),
+                                                (200, 200, 37, 0, 199), (5, 130, 120, 1, 5),
+                                                (2600, 2600, 0, 2045, 2600)])
+def test_indexer_topk_ragged(n, kvl, pos0, rb, re_):
+    cfg = dsa_inputs.custom_config("prefill_4k", n_q=n, n_kv=max(n, kvl), topk=min(2048, 64 + n // 2),
+                                   batch=2, name=f"frag{n}")
+    inp = dsa_inputs.make_inputs(cfg, seed=5)
+    inp["kv_len"][:] = torch.tensor([kvl, max(1, kvl - 9)], dtype=torch.int32)
+    inp["q_pos0"][:] = torch.tensor([pos0, pos0 + 1], dtype=torch.int32)
+    g = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    _assert_same_sets(_fused(cfg, g, rb, re_), _two_pass(cfg, g, rb, re_))
+
+
+def test_indexer_topk_all_ties_take_lowest_indices():
+    """w = 0 makes every visible score exactly 0: the k lowest key indices win."""
+    cfg = dsa_inputs.custom_config("prefill_4k", n_q=3000, n_kv=3000, topk=2048, name="ties")
+    inp = dsa_inputs.make_inputs(cfg, seed=7)
+    inp["w"][:, 2500:] = 0.0
+    g = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    fused = _fused(cfg, g, 2400, 3000)
+    _assert_same_sets(fused, _two_pass(cfg, g, 2400, 3000))
+    got = np.sort(fused.cpu().numpy()[0][100:], axis=-1)
+    assert np.array_equal(got, np.broadcast_to(np.arange(2048, dtype=np.int32), got.shape))
+
+
+def test_indexer_topk_rising_scores_force_compactions():
+    """Positive codes and a key scale that grows with the key index make
+    nearly every new key enter the candidate set: each row's buffer is
+    compacted many times before the end."""
+    cfg = dsa_inputs.custom_config("prefill_4k", n_q=16384, n_kv=16384, topk=2048, name="rise")
+    inp = dsa_inputs.make_inputs(cfg, seed=11)
+    inp["q_fp8"] = inp["q_fp8"] & 0x7F                      # clear the e4m3 sign bit
+    inp["k_fp8"] = inp["k_fp8"] & 0x7F
+    inp["q_fp8"][inp["q_fp8"] == 0x7F] = 0x7E                # no NaN codes
+    inp["k_fp8"][inp["k_fp8"] == 0x7F] = 0x7E
+    inp["w"] = inp["w"].abs()
+    inp["k_scale"] = inp["k_scale"] * (1.0 + torch.arange(cfg.n_kv, dtype=torch.float32) / 64.0)
+    g = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    rb, re_ = cfg.n_q - 256, cfg.n_q
+    _assert_same_sets(_fused(cfg, g, rb, re_), _two_pass(cfg, g, rb, re_))
+
+
 # ------------------------------------------------------------------ attention
 
 def _rand_indices(n_rows, k, n_kv, seed, empty_frac=0.1):
