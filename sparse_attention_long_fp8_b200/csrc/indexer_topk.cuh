@@ -54,7 +54,7 @@ struct IndexerTopkTile {
   static_assert(HI == 64 && DI == 128 && QG == 4, "fused selection is built for H^I=64, d^I=128");
   static constexpr int M = 128;                 // keys per tile (TMEM lanes)
   static constexpr int N = QG * HI;             // MMA N
-  static constexpr int STAGES = 4;
+  static constexpr int STAGES = 3;
   static constexpr int K_BYTES = M * DI;
   static constexpr int Q_BYTES = N * DI;
   static constexpr int EPI_WARPS = 8;
@@ -63,7 +63,7 @@ struct IndexerTopkTile {
   static constexpr uint32_t SWIZZLE = 2u;       // 128-byte rows
   static constexpr uint32_t SBO = 8 * DI;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int CAP = 3968;              // candidates per row
+  static constexpr int CAP = 4480;              // candidates per row
   static constexpr int CHECK_TILES = 4;         // buffers are checked every 4 tiles
   static constexpr int HEADROOM = CHECK_TILES * M;
   static constexpr int MAX_K = 2048;
@@ -395,11 +395,27 @@ struct SelGroup {
       idx_star = ~kth_largest(n, need, [&](int i) { return ~static_cast<uint32_t>(ci[i]); },
                               [&](int i) { return cu[i] == kth; }, &n2, &e2);
     }
-    compact(cu, ci, n,
-            [kth, idx_star](uint32_t u, int32_t ix) {
-              return u > kth || (u == kth && static_cast<uint32_t>(ix) <= idx_star);
-            },
-            out);
+    const auto keep = [kth, idx_star](uint32_t u, int32_t ix) {
+      return u > kth || (u == kth && static_cast<uint32_t>(ix) <= idx_star);
+    };
+    if (out) {
+      // Emit in any order: one pass, slots from warp-aggregated atomics.
+      if (gt == 0) st->above = 0;
+      sync();
+#pragma unroll 4
+      for (int c0 = 0; c0 < n; c0 += 128) {
+        const int i = c0 + gt;
+        const bool take = i < n && keep(cu[i], ci[i]);
+        const uint32_t bal = __ballot_sync(0xffffffffu, take);
+        uint32_t base = 0;
+        if (lane == 0 && bal) base = atomicAdd(&st->above, static_cast<uint32_t>(__popc(bal)));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (take) out[base + __popc(bal & ((1u << lane) - 1u))] = ci[i];
+      }
+      sync();
+    } else {
+      compact(cu, ci, n, keep, nullptr);
+    }
     *kth_out = kth;
     *idx_star_out = idx_star;
   }
