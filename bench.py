@@ -435,11 +435,7 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8e4m3 indexer, bf16 attention, fp32 accumulate",
         "data": "synthetic (seeded; page-shaped workloads)",
-        "config": {"workload": cfg.name, "batch": cfg.batch, "seq_len": cfg.n_q,
-                   "idx_heads": cfg.idx_heads, "idx_dim": cfg.idx_dim, "topk": cfg.topk,
-                   "heads": cfg.heads, "qk_dim": cfg.qk_dim, "v_dim": cfg.v_dim,
-                   "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (q is 9.7 GB per step)"},
+        "config": bench_config(cfg, world),
         "stages_ms": ({"indexer_topk_fused": ix_ms, "attention": at_ms} if fused else
                       {"indexer": ix_ms, "topk": tk_ms, "attention": at_ms}),
         "indexer_tflops_fp8": ix_tf, "indexer_frac_fp8": ix_tf / fp8_peak,
@@ -479,7 +475,13 @@ def main():
                          "ms_per_step": e_ms}
 
     if not args.no_cpu and world == 1 and rank == 0:
-        n_rows = max(16, min(64, os.cpu_count() or 16))
+        # A calibration sample of one row per host thread, then a sample
+        # sized for about 12 s of oracle work.
+        import oracle
+        threads = max(1, oracle.hardware_threads())
+        _, dt0, _, nr0 = oracle_rows_per_s(cfg, seed, threads)
+        reps = max(1, min(32, int(12.0 / max(dt0, 1e-3))))
+        n_rows = min(cfg.n_q, nr0 * reps)
         rps, dt, cores, nr = oracle_rows_per_s(cfg, seed, n_rows)
         result["cpu_baseline"] = {"value": rps * cfg.batch, "unit": "tokens/s", "cores": cores,
                                   "kind": "oracle",
@@ -491,6 +493,15 @@ def main():
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def bench_config(cfg, world):
+    """The workload description both arms print."""
+    return {"workload": cfg.name, "batch": cfg.batch, "seq_len": cfg.n_q,
+            "idx_heads": cfg.idx_heads, "idx_dim": cfg.idx_dim, "topk": cfg.topk,
+            "heads": cfg.heads, "qk_dim": cfg.qk_dim, "v_dim": cfg.v_dim,
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (q is 9.7 GB per step)"}
 
 
 def step_launches_total(stages):
@@ -519,7 +530,7 @@ def main_reference(args, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * sum(secs) / len(secs), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "batch": cfg.batch, "seq_len": cfg.n_q},
+        "config": bench_config(cfg, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
