@@ -553,11 +553,10 @@ __global__ void __launch_bounds__(IndexerTopkTile<HI, DI, QG>::THREADS, 1)
     g.lane = lane;
     const uint32_t k = static_cast<uint32_t>(p.k);
 
-    float cf[T::QPW][HI];
-#pragma unroll
-    for (int q = 0; q < T::QPW; ++q)
-#pragma unroll
-      for (int j = 0; j < HI; ++j) cf[q][j] = coef[(qhalf * T::QPW + q) * HI + j];
+    // The head coefficients stay in shared memory (read as broadcast 16-byte
+    // loads), so that the registers hold both rows' 64 TMEM columns and the
+    // four TMEM loads of a tile are in flight together.
+    const uint32_t coef_addr = smem_u32(coef + qhalf * T::QPW * HI);
 
     uint32_t tau[T::QPW] = {0u, 0u};
     uint32_t tau_idx[T::QPW] = {0xffffffffu, 0xffffffffu};
@@ -571,19 +570,27 @@ __global__ void __launch_bounds__(IndexerTopkTile<HI, DI, QG>::THREADS, 1)
       tc_fence_after();
       const int s = i * T::M + key_local;
       const float ks = s < p.n_kv ? p.k_scale[static_cast<size_t>(b) * p.n_kv + s] : 0.f;
+      uint32_t x[T::QPW][HI];
+      {
+        const uint32_t col = tmem_base + lane_addr + buf * T::N + qhalf * T::QPW * HI;
+#pragma unroll
+        for (int q = 0; q < T::QPW; ++q) {
+          tmem_ld32(col + q * HI, *reinterpret_cast<uint32_t(*)[32]>(&x[q][0]));
+          tmem_ld32(col + q * HI + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[q][32]));
+        }
+        tmem_wait_ld();
+      }
 #pragma unroll
       for (int q = 0; q < T::QPW; ++q) {
         const int ql = qhalf * T::QPW + q;
-        const uint32_t col = tmem_base + lane_addr + buf * T::N + ql * HI;
         float acc = 0.f;
 #pragma unroll
-        for (int h0 = 0; h0 < HI; h0 += 32) {
-          uint32_t x[32];
-          tmem_ld32(col + h0, x);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            acc = fmaf(cf[q][h0 + j], fmaxf(__uint_as_float(x[j]), 0.f), acc);
+        for (int j = 0; j < HI; j += 4) {
+          const uint4 c4 = lds_v4(coef_addr + (q * HI + j) * 4);
+          acc = fmaf(__uint_as_float(c4.x), fmaxf(__uint_as_float(x[q][j]), 0.f), acc);
+          acc = fmaf(__uint_as_float(c4.y), fmaxf(__uint_as_float(x[q][j + 1]), 0.f), acc);
+          acc = fmaf(__uint_as_float(c4.z), fmaxf(__uint_as_float(x[q][j + 2]), 0.f), acc);
+          acc = fmaf(__uint_as_float(c4.w), fmaxf(__uint_as_float(x[q][j + 3]), 0.f), acc);
         }
         const int r = r0 + ql;
         const bool vis = r <= r_last && s < p.n_kv && s <= pos0 + r && s < kvl;
