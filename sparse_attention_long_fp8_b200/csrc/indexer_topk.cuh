@@ -28,8 +28,9 @@
 // to every entry kept.
 //
 // Tile: a CTA owns QG = 4 consecutive query rows and all of their visible key
-// tiles; CTAs are issued longest rows first. Epilogue warps 2-5 own rows 0-1
-// of the group, warps 6-9 rows 2-3 (one TMEM lane quarter each).
+// tiles; CTAs are issued longest rows first. Sixteen epilogue warps, four per
+// SM sub-partition: warps 2-5 own row 0, 6-9 row 1, 10-13 row 2, 14-17 row 3
+// (one TMEM lane quarter each).
 #pragma once
 
 #include "ptx.cuh"
@@ -57,16 +58,18 @@ struct IndexerTopkTile {
   static constexpr int STAGES = 3;
   static constexpr int K_BYTES = M * DI;
   static constexpr int Q_BYTES = N * DI;
-  static constexpr int EPI_WARPS = 8;
+  static constexpr int EPI_WARPS = 16;          // four per SM sub-partition
   static constexpr int THREADS = (2 + EPI_WARPS) * 32;
-  static constexpr int QPW = 2;                 // rows per epilogue warp group
+  static constexpr int QPW = 1;                 // rows per epilogue warp group
+  static constexpr int GROUPS = EPI_WARPS / 4;  // one group of four warps per row
   static constexpr uint32_t SWIZZLE = 2u;       // 128-byte rows
   static constexpr uint32_t SBO = 8 * DI;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int CAP = 4480;              // candidates per row
+  static constexpr int CAP = 4352;              // candidates per row
   static constexpr int CHECK_TILES = 4;         // buffers are checked every 4 tiles
   static constexpr int HEADROOM = CHECK_TILES * M;
   static constexpr int MAX_K = 2048;
+  static_assert(QPW * GROUPS == QG, "one row per warp group");
   static_assert(MAX_K + HEADROOM < CAP, "a compacted buffer must leave room for the next tiles");
   // shared memory carve-up (offsets from a 1024-aligned base)
   static constexpr int OFF_Q = 0;
@@ -76,7 +79,7 @@ struct IndexerTopkTile {
   static constexpr int OFF_CI = OFF_CU + QG * CAP * 4;         // [QG][CAP] key indices
   static constexpr int OFF_SEL = OFF_CI + QG * CAP * 4;        // [2] SelState
   static constexpr int SEL_BYTES = 2048;
-  static constexpr int OFF_BAR = OFF_SEL + 2 * SEL_BYTES;
+  static constexpr int OFF_BAR = OFF_SEL + GROUPS * SEL_BYTES;
   static constexpr int NUM_BARS = 1 + 2 * STAGES + 4;          // q, stages, acc
   static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -542,7 +545,7 @@ __global__ void __launch_bounds__(IndexerTopkTile<HI, DI, QG>::THREADS, 1)
     // ------------------------------------------------------------ epilogue + selection
     const int ew = warp - 2;
     const int quarter = warp & 3;             // TMEM lane quarter this warp may access
-    const int qhalf = ew >> 2;                // rows 2*qhalf, 2*qhalf + 1 of the group
+    const int qhalf = ew >> 2;                // the group: rows QPW*qhalf .. of the CTA's four
     const int key_local = quarter * 32 + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     SelGroup g;
@@ -558,8 +561,12 @@ __global__ void __launch_bounds__(IndexerTopkTile<HI, DI, QG>::THREADS, 1)
     // four TMEM loads of a tile are in flight together.
     const uint32_t coef_addr = smem_u32(coef + qhalf * T::QPW * HI);
 
-    uint32_t tau[T::QPW] = {0u, 0u};
-    uint32_t tau_idx[T::QPW] = {0xffffffffu, 0xffffffffu};
+    uint32_t tau[T::QPW], tau_idx[T::QPW];
+#pragma unroll
+    for (int q = 0; q < T::QPW; ++q) {
+      tau[q] = 0u;
+      tau_idx[q] = 0xffffffffu;
+    }
     // ok turns false when a bounded wait runs out (the error word is set then).
     // The loop still runs to the end, without waiting, appending or writing,
     // so that the group's barriers stay matched.
