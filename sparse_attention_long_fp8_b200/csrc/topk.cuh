@@ -33,7 +33,7 @@ struct TopkParams {
 
 constexpr int kTopkThreads = 1024;
 constexpr int kTopkSamples = 1024;
-constexpr int kTopkCap = 4096;      // candidate buffer (keys + indices: 32 KB)
+constexpr int kTopkCap = 8192;      // candidate buffer (keys + indices: 64 KB)
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   const uint32_t u = __float_as_uint(f + 0.0f);   // -0 -> +0
@@ -152,19 +152,28 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
       (static_cast<int64_t>(5) * p.k * kTopkSamples) / (4 * static_cast<int64_t>(n)) + 8;
   const uint32_t tau = sm.samp[want < kTopkSamples - 1 ? want : kTopkSamples - 1];
 
-  // ---- 2. one pass: candidates >= tau
-  for (int c0 = 0; c0 < n; c0 += kTopkThreads) {
-    const int i = c0 + tid;
-    const uint32_t u = i < n ? order_key(row[i]) : 0u;
-    const bool take = i < n && u >= tau;
-    const uint32_t bal = __ballot_sync(0xffffffffu, take);
-    uint32_t base = 0;
-    if (lane == 0 && bal) base = atomicAdd(&sm.n_cand, static_cast<uint32_t>(__popc(bal)));
-    base = __shfl_sync(0xffffffffu, base, 0);
-    const uint32_t slot = base + __popc(bal & ((1u << lane) - 1u));
-    if (take && slot < static_cast<uint32_t>(kTopkCap)) {
-      sm.cand_u[slot] = u;
-      sm.cand_i[slot] = i;
+  // ---- 2. one pass: candidates >= tau (four independent loads per thread
+  // and round, so the L2 latency of the scores overlaps)
+  for (int c0 = 0; c0 < n; c0 += 4 * kTopkThreads) {
+    uint32_t u[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int i = c0 + tid + m * kTopkThreads;
+      u[m] = i < n ? order_key(row[i]) : 0u;
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int i = c0 + tid + m * kTopkThreads;
+      const bool take = i < n && u[m] >= tau;
+      const uint32_t bal = __ballot_sync(0xffffffffu, take);
+      uint32_t base = 0;
+      if (lane == 0 && bal) base = atomicAdd(&sm.n_cand, static_cast<uint32_t>(__popc(bal)));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      const uint32_t slot = base + __popc(bal & ((1u << lane) - 1u));
+      if (take && slot < static_cast<uint32_t>(kTopkCap)) {
+        sm.cand_u[slot] = u[m];
+        sm.cand_i[slot] = i;
+      }
     }
   }
   __syncthreads();
