@@ -217,6 +217,27 @@ class Step:
         rec("attn")
 
 
+def max_over_ranks(x, dist, device="cuda"):
+    """The max of x over all ranks (x itself without a process group)."""
+    if not dist:
+        return x
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def all_ranks(flag, dist, device="cuda"):
+    """True iff flag holds on every rank: a decision every rank then takes
+    the same way, so that all ranks run the same collectives."""
+    if not dist:
+        return bool(flag)
+    import torch
+    t = torch.tensor([1 if flag else 0], dtype=torch.int32, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MIN)
+    return bool(t.item())
+
+
 def stage_ms(ev):
     """Average per-launch milliseconds and total per stage from event pairs."""
     res = {}
@@ -247,11 +268,7 @@ def timed(step, steps, warmup, dist):
     if dist:
         dist.barrier()
     step.dsa.dsa_check()
-    ms = start.elapsed_time(end) / steps
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(start.elapsed_time(end) / steps, dist)
     return ms, stage_ms(ev)
 
 
@@ -305,11 +322,7 @@ def e2e(cfg, seed, steps, dist):
     e.record()
     torch.cuda.synchronize()
     dsa.dsa_check()
-    ms = s.elapsed_time(e) / steps
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(s.elapsed_time(e) / steps, dist)
     del host, dev, out, lse, idx, h_out, h_lse, h_idx, ws
     torch.cuda.empty_cache()
     return ms, h2d, d2h
@@ -462,12 +475,17 @@ def main():
             del dstep
             torch.cuda.empty_cache()
 
+    # The ranks of a node share its host RAM: every rank needs its own pinned
+    # copy, and all ranks must agree before any of them enters e2e().
     need = e2e_host_bytes(cfg)
     avail = host_available_bytes()
-    if not args.no_e2e and avail is not None and avail < 2 * need:
+    fits = avail is None or avail >= 2 * need * world
+    fits = all_ranks(fits, dist)
+    if not args.no_e2e and not fits:
         result["e2e"] = {"value": None, "unit": "tokens/s",
-                         "skipped": f"host RAM: {avail / 2**30:.0f} GiB available, "
-                                    f"{need / 2**30:.0f} GiB pinned needed"}
+                         "skipped": "host RAM: " + ("unknown" if avail is None else
+                                                    f"{avail / 2**30:.0f} GiB") +
+                                    f" available, {world * need / 2**30:.0f} GiB pinned needed"}
     elif not args.no_e2e:
         e_ms, h2d, d2h = e2e(cfg, seed, max(2, min(args.steps, 3)), dist)
         result["e2e"] = {"value": world * tokens / (e_ms / 1e3), "unit": "tokens/s",

@@ -227,6 +227,16 @@ const char* dsa_last_error(void);
 /* Library version, e.g. "0.1.0". */
 const char* dsa_version(void);
 
+/*
+ * Failure-detection self-test (the paper has no counterpart). Launches one
+ * small kernel that waits, with the same bounded wait every kernel uses, on
+ * a barrier that nothing completes; after limit_ms milliseconds (1..10000)
+ * the wait gives up, sets the device error word and the kernel exits
+ * normally. The next dsa_check() on the stream returns DSA_ERR_TIMEOUT (and
+ * clears the word); the context stays usable. Nothing faults or traps.
+ */
+dsa_status dsa_selftest_wait_timeout(uint32_t limit_ms, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -77,6 +77,8 @@ def load_library(path: str | None = None):
     lib.dsa_forward.argtypes = [SP, P, P, P, P, P, P, P, P, P, P, P, I32, P, P, SZ, P]
     lib.dsa_workspace_size.argtypes = [SP, I32, ctypes.POINTER(SZ)]
     lib.dsa_check.argtypes = [P]
+    lib.dsa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P]
+    lib.dsa_selftest_wait_timeout.restype = ctypes.c_int
     lib.dsa_forward_chunk_rows.argtypes = [SP, ctypes.POINTER(I32)]
     lib.dsa_status_string.argtypes = [ctypes.c_int]
     lib.dsa_status_string.restype = ctypes.c_char_p
@@ -164,6 +166,12 @@ def dsa_indexer_topk(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
         _ptr(w, d["f32"], "w"), _ptr(k_fp8, d["u8"], "k_fp8"), _ptr(k_scale, d["f32"], "k_scale"),
         _ptr(q_pos0, d["i32"], "q_pos0"), _ptr(kv_len, d["i32"], "kv_len"),
         int(row_begin), int(row_end), _ptr(indices, d["i32"], "indices"), _stream(stream)))
+
+
+def dsa_selftest_wait_timeout(limit_ms=100, stream=None):
+    """Launch the bounded-wait self-test; the next dsa_check() raises a
+    DsaError with status DSA_ERR_TIMEOUT."""
+    _raise(load_library().dsa_selftest_wait_timeout(int(limit_ms), _stream(stream)))
 
 
 def dsa_topk(shape, scores, row_begin, row_end, q_pos0, kv_len, indices, ws=None,

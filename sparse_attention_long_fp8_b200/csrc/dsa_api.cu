@@ -19,6 +19,7 @@
 #include "sparse_attn.cuh"
 #include "sparse_attn_vh.cuh"
 #include "topk.cuh"
+#include "selftest.cuh"
 
 namespace {
 
@@ -506,6 +507,17 @@ dsa_status noalloc_scratch_addr(int dev, void** addr) {
 extern "C" {
 
 const char* dsa_version(void) { return "0.1.0"; }
+
+dsa_status dsa_selftest_wait_timeout(uint32_t limit_ms, void* stream) {
+  if (limit_ms == 0 || limit_ms > 10000)
+    return fail(DSA_ERR_INVALID_ARG, "limit_ms must be in [1, 10000] (got %u)", limit_ms);
+  int dev;
+  if (dsa_status st = current_device(&dev)) return st;
+  dsa::wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(limit_ms) * 1000000ull);
+  DSA_CUDA_TRY(cudaGetLastError(), "wait self-test launch");
+  return DSA_OK;
+}
 
 const char* dsa_status_string(dsa_status st) {
   switch (st) {

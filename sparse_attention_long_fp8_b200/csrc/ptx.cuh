@@ -126,6 +126,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// As mbar_wait, with a caller-chosen limit (used by the wait self-test).
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
+                                                unsigned long long limit_ns) {
+  const uint32_t b = smem_u32(bar);
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(b, parity)) return true;
+    if ((it & 63u) == 0 && globaltimer() - t0 > limit_ns) {
+      raise_error(kErrTimeout);
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- proxies
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -68,6 +68,11 @@ def test_indexer_topk_rejects_unsupported_shapes_before_launch(lib):
     assert st == dsa.DSA_ERR_INVALID_ARG
 
 
+def test_selftest_rejects_bad_limit_before_launch(lib):
+    assert lib.dsa_selftest_wait_timeout(0, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_selftest_wait_timeout(10001, None) == dsa.DSA_ERR_INVALID_ARG
+
+
 def test_status_strings(lib):
     for st in range(7):
         assert lib.dsa_status_string(st)
