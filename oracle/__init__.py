@@ -42,6 +42,9 @@ def _load():
         lib.oracle_e4m3_value.restype = ctypes.c_double
         lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
         lib.oracle_hardware_threads.restype = I
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_quantize_rows.argtypes = [ctypes.c_longlong, I, P, P, P]
         lib.oracle_indexer_scores.argtypes = [I, I, I, I, P, P, P, P, P, P, I, P, I]
         lib.oracle_topk.argtypes = [I, I, I, P, P, I]
         lib.oracle_sparse_attn.argtypes = [I, I, I, I, I, I, ctypes.c_double,
@@ -77,6 +80,21 @@ def hardware_threads() -> int:
 
 def e4m3_value(code: int) -> float:
     return float(_load().oracle_e4m3_value(int(code)))
+
+
+def e4m3_encode(v: float) -> int:
+    return int(_load().oracle_e4m3_encode(float(v)))
+
+
+def quantize_rows(x):
+    """Per-row E4M3 encoding of bf16 rows x [rows, dim] (torch bf16 or raw
+    uint16 bits): returns (codes uint8 [rows, dim], scales float32 [rows])."""
+    xb = _np(x, np.uint16)
+    rows, dim = xb.shape
+    codes = np.zeros((rows, dim), dtype=np.uint8)
+    scales = np.zeros(rows, dtype=np.float32)
+    _load().oracle_quantize_rows(rows, dim, _ptr(xb), _ptr(codes), _ptr(scales))
+    return codes, scales
 
 
 def indexer_scores(q8, qs, w, k8, ks, pos, kv_len, n_threads=0):

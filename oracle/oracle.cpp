@@ -11,6 +11,8 @@
 //   * fine-grained token selection, equation u_t = Attn(h_t, {c_s | I_{t,s}
 //     in Top-k(I_{t,:})}): the k keys with the largest score, ties broken by
 //     the lower key index, fewer than k valid keys -> all of them, pad -1;
+//   * the per-row FP8 encoding of the indexer inputs (scale = amax / 448,
+//     nearest E4M3 value, ties to even, saturating);
 //   * the attention over the selected latent rows c_s (MQA: every query head
 //     reads the same row; K = all qk_dim dims, V = the first v_dim dims; the
 //     latent width 576 = 512 + 64 follows the MLA section 1.1 of page
@@ -48,6 +50,27 @@ double e4m3_value(uint8_t code) {
   return sign ? -mag : mag;
 }
 
+// Encode a float into E4M3 "fn" by the definition: the finite code whose
+// value is nearest to v (exact comparison in fp64), ties to the code with an
+// even mantissa, magnitudes at or above 448 saturating to +-448, the sign of v
+// (including -0) kept in bit 7. A NaN maps to the NaN code 0x7F.
+uint8_t e4m3_encode(float v) {
+  if (std::isnan(v)) return 0x7F;
+  const uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+  const double a = std::fabs(static_cast<double>(v));
+  if (a >= 448.0) return sign | 0x7E;
+  uint8_t best = 0;
+  double best_d = std::numeric_limits<double>::infinity();
+  for (int c = 0; c <= 0x7E; ++c) {   // every non-negative finite code
+    const double d = std::fabs(a - e4m3_value(static_cast<uint8_t>(c)));
+    if (d < best_d || (d == best_d && (c & 1) == 0)) {
+      best_d = d;
+      best = static_cast<uint8_t>(c);
+    }
+  }
+  return sign | best;
+}
+
 // bfloat16 is the upper half of an IEEE binary32.
 double bf16_value(uint16_t bits) {
   uint32_t u = static_cast<uint32_t>(bits) << 16;
@@ -83,6 +106,30 @@ int oracle_hardware_threads() {
 }
 
 double oracle_e4m3_value(uint8_t code) { return e4m3_value(code); }
+
+uint8_t oracle_e4m3_encode(float v) { return e4m3_encode(v); }
+
+// Per-row FP8 quantisation of bf16 rows (the indexer's inputs: one scale per
+// row of d^I values, scale = amax / 448, amax = 0 -> scale 1). The scale and
+// each x / scale are computed in fp32 (the precision the GPU kernel decides
+// the codes in); the code is then the definition's nearest E4M3 value.
+//   x [rows, dim] bf16 bits -> codes [rows, dim], scales [rows]
+void oracle_quantize_rows(long long rows, int dim, const uint16_t* x, uint8_t* codes,
+                          float* scales) {
+  for (long long r = 0; r < rows; ++r) {
+    const uint16_t* xr = x + r * dim;
+    float amax = 0.0f;
+    for (int d = 0; d < dim; ++d)
+      amax = std::max(amax, std::fabs(static_cast<float>(bf16_value(xr[d]))));
+    const float scale = amax > 0.0f ? amax / 448.0f : 1.0f;
+    scales[r] = scale;
+    for (int d = 0; d < dim; ++d) {
+      float y = static_cast<float>(bf16_value(xr[d])) / scale;
+      y = std::min(448.0f, std::max(-448.0f, y));
+      codes[r * dim + d] = e4m3_encode(y);
+    }
+  }
+}
 
 // Indexer scores for n_rows query rows of ONE sequence.
 //   q8   [n_rows, HI, DI] e4m3 codes,  qs [n_rows, HI] scale per (row, head)

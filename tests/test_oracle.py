@@ -70,6 +70,82 @@ def test_e4m3_exhaustive_vs_torch(oracle_lib):
 
 # ---------------------------------------------------------------- indexer
 
+def _finite_codes():
+    return [c for c in range(256) if (c & 0x7F) != 0x7F]
+
+
+def test_e4m3_encode_round_trips_every_finite_code(oracle_lib):
+    """Encoding a code's own value gives the code back (sign of zero kept)."""
+    for c in _finite_codes():
+        v = oracle_lib.e4m3_value(c)
+        assert oracle_lib.e4m3_encode(v if c != 0x80 else -0.0) == c
+
+
+def test_e4m3_encode_ties_go_to_even_mantissa(oracle_lib):
+    """Exactly half-way between two adjacent codes (exact in fp32) the code
+    with the even mantissa wins; a hair either side picks the nearer one."""
+    for c in range(0x00, 0x7E):
+        lo, hi = oracle_lib.e4m3_value(c), oracle_lib.e4m3_value(c + 1)
+        mid = np.float32((lo + hi) / 2)
+        assert float(mid) == (lo + hi) / 2
+        even = c if c % 2 == 0 else c + 1
+        assert oracle_lib.e4m3_encode(float(mid)) == even
+        assert oracle_lib.e4m3_encode(-float(mid)) == (0x80 | even)
+        below = np.nextafter(mid, np.float32(-np.inf), dtype=np.float32)
+        above = np.nextafter(mid, np.float32(np.inf), dtype=np.float32)
+        assert oracle_lib.e4m3_encode(float(below)) == c
+        assert oracle_lib.e4m3_encode(float(above)) == c + 1
+
+
+def test_e4m3_encode_saturates(oracle_lib):
+    for v, want in [(448.0, 0x7E), (460.0, 0x7E), (1e30, 0x7E), (-449.0, 0xFE), (-1e30, 0xFE)]:
+        assert oracle_lib.e4m3_encode(v) == want
+
+
+def test_e4m3_encode_matches_library_cast(oracle_lib):
+    """Library special case: torch's round-to-nearest-even float8_e4m3fn cast,
+    after clamping to the finite range, on a dense sweep of fp32 values."""
+    g = torch.Generator().manual_seed(3)
+    v = torch.cat([torch.randn(20000, generator=g) * 100,
+                   torch.randn(5000, generator=g) * 1e-2,
+                   torch.linspace(-460, 460, 9201)]).float()
+    ref = v.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle_lib.e4m3_encode(float(x)) for x in v.numpy()], dtype=np.uint8)
+    assert np.array_equal(got, ref)
+
+
+def test_quantize_rows_scale_and_extremes(oracle_lib):
+    """Per row: scale = amax / 448 in fp32, the amax element encodes to the
+    extreme code, a zero row gets scale 1 and zero codes, and decoding
+    (code value * scale) is within half an E4M3 step of x."""
+    g = torch.Generator().manual_seed(5)
+    x = (torch.randn(6, 128, generator=g) * torch.tensor([1, 1e-3, 50, 1, 1, 0]).view(6, 1))
+    x = x.to(torch.bfloat16)
+    codes, scales = oracle_lib.quantize_rows(x)
+    xf = x.float().numpy()
+    for r in range(6):
+        amax = np.float32(np.abs(xf[r]).max())
+        if amax == 0:
+            assert scales[r] == 1.0 and ((codes[r] & 0x7F) == 0).all()   # +-0 keep their sign
+            continue
+        assert scales[r] == np.float32(amax / np.float32(448.0))
+        j = int(np.abs(xf[r]).argmax())
+        assert codes[r, j] in (0x7E, 0xFE)
+        dec = np.array([oracle_lib.e4m3_value(int(c)) for c in codes[r]]) * scales[r]
+        # relative E4M3 step is 2^-3 for normals; absolute floor at the subnormal step
+        tol = np.maximum(np.abs(xf[r]) * 2.0 ** -4, 2.0 ** -10 * scales[r]) * 1.0001
+        assert (np.abs(dec - xf[r]) <= tol).all()
+
+
+def test_quantize_rows_matches_library_encoding(oracle_lib):
+    """Library special case: torch's amax / 448, fp32 division and RNE cast."""
+    g = torch.Generator().manual_seed(7)
+    x = (torch.randn(64, 128, generator=g) * torch.rand(64, 1, generator=g) * 10).to(torch.bfloat16)
+    codes, scales = oracle_lib.quantize_rows(x)
+    tc, ts = dsa_inputs.quantize_e4m3_rows(x)
+    assert np.array_equal(codes, tc.numpy()) and np.array_equal(scales, ts.numpy())
+
+
 def test_indexer_single_head_is_relu_matmul(oracle_lib):
     """H^I = 1, w = 1, unit scales: I[t,s] = ReLU(q_t . k_s), a plain matmul."""
     n, S, DI = 9, 13, 32
