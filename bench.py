@@ -238,6 +238,45 @@ def all_ranks(flag, dist, device="cuda"):
     return bool(t.item())
 
 
+def quantiser_bench(cfg, peaks, reps=10):
+    """The per-row FP8 quantiser on the workload's indexer inputs (bf16
+    q [T, H^I, d^I] and k [S, d^I]); HBM-bound: 3 bytes per element plus a
+    scale per row. Inputs (2.2 GB at 64K) exceed L2."""
+    import torch
+    import sparse_attention_long_fp8_b200 as dsa
+    g = torch.Generator(device="cuda").manual_seed(5)
+    xs = [torch.randn(cfg.batch * cfg.n_q, cfg.idx_heads, cfg.idx_dim, device="cuda", generator=g,
+                      dtype=torch.bfloat16),
+          torch.randn(cfg.batch * cfg.n_kv, cfg.idx_dim, device="cuda", generator=g,
+                      dtype=torch.bfloat16)]
+    outs = [(torch.empty(x.shape, dtype=torch.uint8, device="cuda"),
+             torch.empty(x.shape[:-1], device="cuda")) for x in xs]
+    nbytes = sum(x.numel() * 3 + x.numel() // x.shape[-1] * 4 for x in xs)
+
+    def run():
+        for x, (c, sc) in zip(xs, outs):
+            dsa.dsa_quantize_e4m3(x, c, sc)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    dsa.dsa_check()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(reps):
+        run()
+    e.record()
+    torch.cuda.synchronize()
+    dsa.dsa_check()
+    ms = s.elapsed_time(e) / reps
+    gbs = nbytes / (ms / 1e3) / 1e9
+    del xs, outs
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "GB_per_s": gbs, "frac_hbm": gbs / peaks["hbm"],
+            "algorithmic_bytes": nbytes, "launches": 2,
+            "what": "q [T*H^I, d^I] and k [S, d^I] bf16 -> e4m3 codes + fp32 row scales"}
+
+
 def stage_ms(ev):
     """Average per-launch milliseconds and total per stage from event pairs."""
     res = {}
@@ -456,6 +495,9 @@ def main():
         "roofline": roof, "gpu_launches": step_launches_total(stages),
         "clocks": clock_info,
     }
+
+    if not args.no_decode:
+        result["quantiser"] = quantiser_bench(cfg, peaks)
 
     if not args.no_decode:
         result["decode"] = {}

@@ -101,6 +101,23 @@ dsa_status dsa_indexer_scores(const dsa_shape* shape, const uint8_t* q_fp8,
                               int32_t flags, float* scores, void* stream);
 
 /*
+ * Per-row FP8 quantisation of the indexer inputs (page "DeepseekV3.2 拆解",
+ * section "闪电索引器": the indexer computes in FP8). For each row r of dim
+ * values: scale[r] = amax_r / 448 (1 when the row is all zero), and
+ * codes[r, d] = E4M3(clamp(x[r, d] / scale[r], -448, 448)) rounded to
+ * nearest even (saturating, sign of zero kept). scale and x / scale are
+ * fp32 IEEE operations, so the codes are reproducible bit for bit.
+ *   x      [rows, dim] bf16 (raw bits)   (2 * dim / 32 -byte aligned)
+ *   codes  [rows, dim] e4m3fn codes      (dim / 32 -byte aligned)
+ *   scales [rows] fp32
+ * The indexer's q_fp8 / q_scale are the rows of [B, T, H^I, d^I] (one scale
+ * per token and head) and k_fp8 / k_scale those of [B, S, d^I]. dim must be
+ * 32, 64 or 128 (DSA_ERR_UNSUPPORTED otherwise); rows = 0 launches nothing.
+ */
+dsa_status dsa_quantize_e4m3(int64_t rows, int32_t dim, const uint16_t* x, uint8_t* codes,
+                             float* scales, void* stream);
+
+/*
  * Indexer scores and top-k selection in one kernel (page "DeepseekV3.2 拆解",
  * section "闪电索引器", eq. I_{t,s}, and section "细粒度 Token 选择机制",
  * eq. u_t). Inputs and row range as dsa_indexer_scores; the score of each

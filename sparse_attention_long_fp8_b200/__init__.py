@@ -77,6 +77,8 @@ def load_library(path: str | None = None):
     lib.dsa_forward.argtypes = [SP, P, P, P, P, P, P, P, P, P, P, P, I32, P, P, SZ, P]
     lib.dsa_workspace_size.argtypes = [SP, I32, ctypes.POINTER(SZ)]
     lib.dsa_check.argtypes = [P]
+    lib.dsa_quantize_e4m3.argtypes = [ctypes.c_int64, I32, P, P, P, P]
+    lib.dsa_quantize_e4m3.restype = ctypes.c_int
     lib.dsa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P]
     lib.dsa_selftest_wait_timeout.restype = ctypes.c_int
     lib.dsa_forward_chunk_rows.argtypes = [SP, ctypes.POINTER(I32)]
@@ -166,6 +168,23 @@ def dsa_indexer_topk(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
         _ptr(w, d["f32"], "w"), _ptr(k_fp8, d["u8"], "k_fp8"), _ptr(k_scale, d["f32"], "k_scale"),
         _ptr(q_pos0, d["i32"], "q_pos0"), _ptr(kv_len, d["i32"], "kv_len"),
         int(row_begin), int(row_end), _ptr(indices, d["i32"], "indices"), _stream(stream)))
+
+
+def dsa_quantize_e4m3(x, codes, scales, stream=None):
+    """Per-row E4M3 quantisation of a bf16 tensor x [..., dim] into codes
+    (uint8, same shape) and scales (fp32, x.shape[:-1])."""
+    import torch
+    d = _dt()
+    rows = x.numel() // x.shape[-1] if x.numel() else 0
+    if codes.shape != x.shape or tuple(scales.shape) != tuple(x.shape[:-1]):
+        raise ValueError("codes must match x and scales must be x.shape[:-1]")
+    for t, name in ((x, "x"), (codes, "codes"), (scales, "scales")):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    _raise(load_library().dsa_quantize_e4m3(
+        int(rows), int(x.shape[-1]), _ptr(x, d["bf16"], "x"),
+        _ptr(codes, (torch.uint8, torch.float8_e4m3fn), "codes"), _ptr(scales, d["f32"], "scales"),
+        _stream(stream)))
 
 
 def dsa_selftest_wait_timeout(limit_ms=100, stream=None):

@@ -20,6 +20,7 @@
 #include "sparse_attn_vh.cuh"
 #include "topk.cuh"
 #include "selftest.cuh"
+#include "quantize.cuh"
 
 namespace {
 
@@ -507,6 +508,33 @@ dsa_status noalloc_scratch_addr(int dev, void** addr) {
 extern "C" {
 
 const char* dsa_version(void) { return "0.1.0"; }
+
+dsa_status dsa_quantize_e4m3(int64_t rows, int32_t dim, const uint16_t* x, uint8_t* codes,
+                             float* scales, void* stream) {
+  if (rows < 0) return fail(DSA_ERR_INVALID_ARG, "rows must be >= 0 (got %lld)", static_cast<long long>(rows));
+  if (dim != 32 && dim != 64 && dim != 128)
+    return fail(DSA_ERR_UNSUPPORTED, "dsa_quantize_e4m3 supports dim 32, 64, 128 (got %d)", dim);
+  if (dsa_status st = check_ptrs({x, codes, scales}, "dsa_quantize_e4m3")) return st;
+  const int per = dim / 32;
+  if (!aligned(x, 2 * per) || !aligned(codes, per) || !aligned(scales, 4))
+    return fail(DSA_ERR_INVALID_ARG, "x must be %d-byte and codes %d-byte aligned", 2 * per, per);
+  const long long blocks = (rows + dsa::kQuantRowsPerCta - 1) / dsa::kQuantRowsPerCta;
+  if (blocks >= (1ll << 31)) return fail(DSA_ERR_INVALID_ARG, "too many rows");
+  if (rows == 0) return DSA_OK;
+  int dev;
+  if (dsa_status st = current_device(&dev)) return st;
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  const unsigned grid = static_cast<unsigned>(blocks);
+  constexpr int threads = 32 * dsa::kQuantWarps;
+  if (per == 4)
+    dsa::quantize_e4m3_rows_kernel<4><<<grid, threads, 0, st_>>>(x, codes, scales, rows);
+  else if (per == 2)
+    dsa::quantize_e4m3_rows_kernel<2><<<grid, threads, 0, st_>>>(x, codes, scales, rows);
+  else
+    dsa::quantize_e4m3_rows_kernel<1><<<grid, threads, 0, st_>>>(x, codes, scales, rows);
+  DSA_CUDA_TRY(cudaGetLastError(), "quantiser launch");
+  return DSA_OK;
+}
 
 dsa_status dsa_selftest_wait_timeout(uint32_t limit_ms, void* stream) {
   if (limit_ms == 0 || limit_ms > 10000)

@@ -73,6 +73,14 @@ def test_selftest_rejects_bad_limit_before_launch(lib):
     assert lib.dsa_selftest_wait_timeout(10001, None) == dsa.DSA_ERR_INVALID_ARG
 
 
+def test_quantiser_argument_checks(lib):
+    assert lib.dsa_quantize_e4m3(16, 96, FAKE, FAKE, FAKE, None) == dsa.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_quantize_e4m3(-1, 128, FAKE, FAKE, FAKE, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_quantize_e4m3(16, 128, None, FAKE, FAKE, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_quantize_e4m3(16, 128, FAKE + 2, FAKE, FAKE, None) == dsa.DSA_ERR_INVALID_ARG
+    assert lib.dsa_quantize_e4m3(0, 128, FAKE, FAKE, FAKE, None) == dsa.DSA_OK
+
+
 def test_status_strings(lib):
     for st in range(7):
         assert lib.dsa_status_string(st)
