@@ -20,7 +20,14 @@
 // logit MMAs of a block run over the logit-only part first, so the gather of
 // block i + 2 overlaps S(i + 1) and PV(i).
 //
-// TMEM per CTA: O 256 columns, S 64, P 32, Q 160 = 512.
+// S is double-buffered in TMEM, and P(i) (bf16, 32 columns) is written over
+// the first half of S(i)'s own buffer once both softmax warps of a lane
+// quarter have read it. S(i + 1) is issued as soon as PV(i - 1) has released
+// its buffer, so the tensor pipe does not wait for the softmax to read S(i).
+//
+// TMEM per CTA: O 256 columns, S 2 x 64, Q 128 (four logit-only dim blocks)
+// = 512. Q's other five dim blocks (the V half and the RoPE block) are in
+// shared memory.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -42,27 +49,33 @@ struct VhTile {
   static constexpr int DB_BYTES = NK * 128;     // one 64-dim block of a stage
   static constexpr int STAGE_BYTES = NDB * DB_BYTES;
   static constexpr int STAGES = 2;
-  static constexpr int QS_BYTES = VDB * M * 128;
+  static constexpr int XT = 4;                  // logit-only Q blocks held in TMEM
+  static constexpr int QSB = VDB + 1;           // Q blocks in shared memory: V half + RoPE
+  static constexpr int QS_BYTES = QSB * M * 128;
   static constexpr int PRODUCERS = 128;
   static constexpr int THREADS = 448;           // gather 0-3, S MMA 4, softmax 5-12, PV MMA 13
   static constexpr int SOFTMAX_WARPS = 8;       // two per TMEM lane quarter, 32 keys each
-  static constexpr int COL_O = 0, COL_S = 256, COL_P = 320, COL_Q = 352;
+  static constexpr int COL_O = 0, COL_S = 256, COL_Q = 384;   // S buffer b at COL_S + 64 b
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int OFF_C = 0;
   static constexpr int OFF_QS = STAGES * STAGE_BYTES;
   static constexpr int OFF_RED = OFF_QS + QS_BYTES;          // [2 parity][2 halves][128] fp32
-  static constexpr int OFF_END = OFF_RED + 2 * 2 * M * 4;    // [half][l, l_mma][128] fp32
-  static constexpr int OFF_BAR = OFF_END + 2 * 2 * M * 4;
-  static constexpr int NUM_BARS = 4 * STAGES + 5 + 8 + 4;    // stages, singles, red[8], end[4]
-  static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
+  static constexpr int OFF_END = OFF_C;      // [half][l, l_mma][128] fp32, after the last PV
+  static constexpr int OFF_BAR = OFF_RED + 2 * 2 * M * 4;
+  static constexpr int NUM_BARS = 4 * STAGES + 6 + 8 + 4;    // stages, singles, red[8], end[4]
+  // No alignment slack: the dynamic shared memory of this kernel starts on a
+  // 1024-byte boundary (checked at run time; a misaligned base is reported).
+  static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   static_assert(STAGE_BYTES % 1024 == 0 && OFF_QS % 1024 == 0, "1024-byte aligned operands");
-  static_assert(COL_Q + XDB * 32 == 512, "TMEM columns");
+  static_assert(COL_Q + XT * 32 == 512, "TMEM columns");
 };
 
-// Latent dim block of the t-th logit-only block of V-half v (t = 0..4): the
-// other half's four value blocks, then the RoPE block 8.
-__device__ __forceinline__ int vh_xblock(int t, int v) { return t == 4 ? 8 : t + 4 * (1 - v); }
+// Latent dim block of the t-th Q block held in TMEM (t = 0..3): the other
+// half's four value blocks. The u-th Q block in shared memory (u = 0..4) is
+// block 4v + u of this CTA's value half, then the RoPE block 8.
+__device__ __forceinline__ int vh_tblock(int t, int v) { return t + 4 * (1 - v); }
+__device__ __forceinline__ int vh_sblock(int u, int v) { return u == 4 ? 8 : 4 * v + u; }
 
 // Warp roles: 0-3 gather (cp.async, 16 bytes per copy); 4 issues
 // the logit MMAs and owns TMEM; 5-12 run the softmax (two warps per TMEM lane
@@ -80,15 +93,18 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
   uint64_t* cv_full = bars + T::STAGES;          // [2] V-half blocks landed
   uint64_t* cx_empty = bars + 2 * T::STAGES;     // [2] S of the stage's block finished
   uint64_t* cv_empty = bars + 3 * T::STAGES;     // [2] PV of the stage's block finished
-  uint64_t* s_full = bars + 4 * T::STAGES;       // S tile written
-  uint64_t* s_free = s_full + 1;                 // S tile read by the softmax warps
-  uint64_t* p_full = s_full + 2;                 // P tile written
-  uint64_t* pv_done = s_full + 3;                // PV finished (P tile free, O updated)
-  uint64_t* q_ready = s_full + 4;                // Q in TMEM and shared memory
-  uint64_t* red_bar = s_full + 5;                // [parity][quarter]: both half maxima written
-  uint64_t* end_bar = s_full + 13;               // [quarter]: both halves of l, l_mma written
+  uint64_t* s_full = bars + 4 * T::STAGES;       // [2] S tile of buffer b written
+  uint64_t* pv_done = s_full + 2;                // [2] PV of buffer b finished (buffer free, O updated)
+  uint64_t* p_full = s_full + 4;                 // P tile written
+  uint64_t* q_ready = s_full + 5;                // Q in TMEM and shared memory
+  uint64_t* red_bar = s_full + 6;                // [parity][quarter]: both half maxima written
+  uint64_t* end_bar = s_full + 14;               // [quarter]: both halves of l, l_mma written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + T::NUM_BARS);
 
+  if ((smem_u32(smem_raw) & 1023u) != 0) {      // see SMEM_BYTES: no slack to realign
+    if (threadIdx.x == 0) raise_error(kErrInternal);
+    return;
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int vh = blockIdx.x & 1;                 // value half of this CTA
@@ -109,10 +125,11 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
       mbar_init(&cx_empty[s], 1);
       mbar_init(&cv_empty[s], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_free, T::SOFTMAX_WARPS);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&pv_done[s], 1);
+    }
     mbar_init(p_full, T::SOFTMAX_WARPS);
-    mbar_init(pv_done, 1);
     mbar_init(q_ready, T::SOFTMAX_WARPS);
     for (int s = 0; s < 12; ++s) mbar_init(&red_bar[s], 2);
     fence_mbar_init();
@@ -204,38 +221,46 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
     for (int i = 0; i < n_blocks && ok; ++i) {
       const int st = i % T::STAGES;
       const uint32_t ph = (i / T::STAGES) & 1;
-      ok = mbar_wait(s_free, (i & 1) ^ 1) && mbar_wait(&cx_full[st], ph);
+      const int sb = i & 1;                            // S buffer of block i
+      // buffer sb is free once PV(i - 2) has read the P it held
+      ok = mbar_wait(&pv_done[sb], ((i >> 1) & 1) ^ 1) && mbar_wait(&cx_full[st], ph);
       if (!ok) break;
       fence_proxy_async_smem();
       tc_fence_after();
+      const uint32_t d_s = tmem_base + T::COL_S + sb * T::NK;
       const uint64_t cd = c_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
-      // logit-only blocks (the other half's value blocks, then RoPE block 8),
-      // Q slice from TMEM
+      // logit-only part of the stage: the other half's value blocks with Q
+      // from TMEM, then the RoPE block with Q from shared memory
 #pragma unroll
-      for (int t = 0; t < T::XDB; ++t)
+      for (int t = 0; t < T::XT; ++t)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = t < 4 ? cd + x_shift + ((t * T::DB_BYTES + kk * 32) >> 4)
-                                    : cd + ((8 * T::DB_BYTES + kk * 32) >> 4);
+          const uint64_t bd = cd + x_shift + ((t * T::DB_BYTES + kk * 32) >> 4);
           if (elect_one())
-            umma_bf16_ts(tmem_base + T::COL_S, tmem_base + T::COL_Q + t * 32 + kk * 8, bd,
-                         idesc_s, (t | kk) ? 1u : 0u);
+            umma_bf16_ts(d_s, tmem_base + T::COL_Q + t * 32 + kk * 8, bd, idesc_s,
+                         (t | kk) ? 1u : 0u);
         }
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = q_desc0 + ((4 * T::M * 128 + kk * 32) >> 4);
+        const uint64_t bd = cd + ((8 * T::DB_BYTES + kk * 32) >> 4);
+        if (elect_one()) umma_bf16_ss(d_s, ad, bd, idesc_s, 1u);
+      }
       if (elect_one()) umma_commit(&cx_empty[st]);
       ok = mbar_wait(&cv_full[st], ph);
       if (!ok) break;
       fence_proxy_async_smem();
       tc_fence_after();
-      // V-half blocks, Q slice from shared memory
+      // V-half blocks, Q from shared memory
 #pragma unroll
       for (int u = 0; u < T::VDB; ++u)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t ad = q_desc0 + ((u * T::M * 128 + kk * 32) >> 4);
           const uint64_t bd = cd + v_shift + ((u * T::DB_BYTES + kk * 32) >> 4);
-          if (elect_one()) umma_bf16_ss(tmem_base + T::COL_S, ad, bd, idesc_s, 1u);
+          if (elect_one()) umma_bf16_ss(d_s, ad, bd, idesc_s, 1u);
         }
-      if (elect_one()) umma_commit(s_full);
+      if (elect_one()) umma_commit(&s_full[sb]);
     }
     __syncwarp();
   } else if (warp == 13) {
@@ -248,16 +273,18 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
       if (!mbar_wait(p_full, j & 1)) break;
       tc_fence_after();
       // P(j) exists only after S(j) was read, so S(j) has completed: when
-      // PV(j) completes, both readers of the V-half blocks are done.
+      // PV(j) completes, both readers of the V-half blocks are done, and the
+      // S / P buffer of block j is free.
       const uint64_t vd = v_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
+      const uint32_t a_p = tmem_base + T::COL_S + (j & 1) * T::NK;   // P over S's first half
 #pragma unroll
       for (int kk = 0; kk < NK / 16; ++kk)
         if (elect_one())
-          umma_bf16_ts(tmem_base + T::COL_O, tmem_base + T::COL_P + kk * 8,
-                       vd + ((kk * 2048) >> 4), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem_base + T::COL_O, a_p + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv,
+                       (j > 0 || kk > 0) ? 1u : 0u);
       if (elect_one()) {
         umma_commit(&cv_empty[st]);
-        umma_commit(pv_done);
+        umma_commit(&pv_done[j & 1]);
       }
     }
     __syncwarp();
@@ -269,15 +296,15 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     float* red = reinterpret_cast<float*>(smem + T::OFF_RED);   // [parity][half][128]
 
-    // Q into TMEM (logit-only blocks; the two warps of a quarter take
-    // alternate 16-column chunks) and shared memory (V-half blocks, K-major
-    // 128-byte swizzle; each warp writes two of the four blocks).
+    // Q into TMEM (four logit-only blocks; the two warps of a quarter take
+    // alternate 16-column chunks) and shared memory (V-half blocks and the
+    // RoPE block, K-major 128-byte swizzle; the two warps alternate blocks).
     {
       const __nv_bfloat16* qh = p.q + (static_cast<size_t>(row) * p.H + min(h, p.H - 1)) * T::DQK;
       const bool live = h < p.H;
-      for (int c = half; c < T::XDB * 2; c += 2) {
+      for (int c = half; c < T::XT * 2; c += 2) {
         uint32_t v[16];
-        const uint4* src = reinterpret_cast<const uint4*>(qh + vh_xblock(c >> 1, vh) * 64 + (c & 1) * 32);
+        const uint4* src = reinterpret_cast<const uint4*>(qh + vh_tblock(c >> 1, vh) * 64 + (c & 1) * 32);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const uint4 u = live ? src[k] : make_uint4(0u, 0u, 0u, 0u);
@@ -285,8 +312,8 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
         }
         tmem_st16(tmem_base + lane_addr + T::COL_Q + c * 16, v);
       }
-      for (int u = 2 * half; u < 2 * half + 2; ++u) {
-        const uint4* src = reinterpret_cast<const uint4*>(qh + (4 * vh + u) * 64);
+      for (int u = half; u < T::QSB; u += 2) {
+        const uint4* src = reinterpret_cast<const uint4*>(qh + vh_sblock(u, vh) * 64);
         uint8_t* dst = qs_smem + u * (T::M * 128) + (h >> 3) * 1024 + (h & 7) * 128;
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch)
@@ -312,17 +339,15 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
     uint32_t sr[32];
     float z[32];
     for (int i = 0; i < n_blocks && ok; ++i) {
-      // ---- logits of this warp's 32 keys; the S tile is free for S(i + 1)
+      // ---- logits of this warp's 32 keys from S buffer i & 1
       const int idx = idx_next;
       idx_next = load_idx(i + 1);
       const uint32_t vmask = __ballot_sync(0xffffffffu, idx >= 0 && idx < p.n_kv);
-      if (!(ok = mbar_wait(s_full, i & 1))) break;
+      const uint32_t col_s = T::COL_S + (i & 1) * T::NK;
+      if (!(ok = mbar_wait(&s_full[i & 1], (i >> 1) & 1))) break;
       tc_fence_after();
-      tmem_ld32(tmem_base + lane_addr + T::COL_S + half * 32, sr);
+      tmem_ld32(tmem_base + lane_addr + col_s + half * 32, sr);
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
       // ---- block max over the 64 keys, shared with the partner warp
       float hmax = -INFINITY;
 #pragma unroll
@@ -332,16 +357,20 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
       }
       float* red_i = red + (i & 1) * (2 * T::M);
       red_i[half * T::M + h] = hmax;
+      // After this exchange both warps of the quarter have read their S
+      // columns, so P may overwrite the buffer's first 32 columns.
+      tc_fence_before();
       __syncwarp();
       uint64_t* rb = &red_bar[(i & 1) * 4 + quarter];
       if (lane == 0) mbar_arrive(rb);
       if (!(ok = mbar_wait(rb, (i >> 1) & 1))) break;
+      tc_fence_after();
       const float bmax = fmaxf(hmax, red_i[(half ^ 1) * T::M + h]);
       // ---- online softmax; P(i) into TMEM once PV(i - 1) has finished
       const bool grow = bmax > m_used + 8.0f;
       const float m_new = grow ? bmax : m_used;
       if (i > 0) {
-        if (!(ok = mbar_wait(pv_done, (i - 1) & 1))) break;
+        if (!(ok = mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1))) break;
         tc_fence_after();
       }
       if (i > 0 && __any_sync(0xffffffffu, grow)) {
@@ -379,17 +408,18 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
       }
       l += lsum;
       l_mma += lsum_mma;
-      tmem_st16(tmem_base + lane_addr + T::COL_P + half * 16, pk);
+      tmem_st16(tmem_base + lane_addr + col_s + half * 16, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
     }
     if (ok && n_blocks > 0) {
-      ok = mbar_wait(pv_done, (n_blocks - 1) & 1);
+      ok = mbar_wait(&pv_done[(n_blocks - 1) & 1], ((n_blocks - 1) >> 1) & 1);
       tc_fence_after();
     }
-    // Both warps of a quarter add their halves of l and l_mma.
+    // Both warps of a quarter add their halves of l and l_mma (through the
+    // stage area: every gather and MMA has finished by now).
     float* red_l = reinterpret_cast<float*>(smem + T::OFF_END);   // [half][2][128]
     red_l[(half * 2) * T::M + h] = l;
     red_l[(half * 2 + 1) * T::M + h] = l_mma;
