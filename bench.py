@@ -467,9 +467,16 @@ def main():
     dominant = max(("indexer", ix_ms), ("attn", at_ms), ("topk", tk_ms), key=lambda x: x[1])[0]
     ix_kernel = "indexer_topk_kernel<64,128,4>" if fused else "indexer_scores_kernel<64,128,4>"
     if dominant == "attn":
+        # DRAM bytes of sparse_attn_vh_kernel from one ncu capture at L = 4096
+        # (dram__bytes_read.sum + dram__bytes_write.sum = 642.5 MB + 1022.6 MB,
+        # profiles/ncu_full_prefill_4k.md); its traffic grows in proportion to
+        # the query rows, so it is scaled by rows. Re-capture when the kernel
+        # changes.
+        traffic = (642.484736e6 + 1022.602e6) / 4096 * cfg.batch * cfg.n_q
         roof = {"kernel": "sparse_attn_vh_kernel", "bound": "tensor",
                 "achieved": at_f / (at_ms / 1e3) / 1e12, "peak": peaks["bf16_sustained"],
-                "unit": "TFLOP/s", "traffic": None}
+                "unit": "TFLOP/s", "traffic": traffic,
+                "traffic_source": "ncu DRAM bytes of one 4096-row launch, scaled by rows"}
     elif dominant == "indexer":
         roof = {"kernel": ix_kernel, "bound": "tensor",
                 "achieved": ix_tf, "peak": fp8_peak, "unit": "TFLOP/s", "traffic": None}
