@@ -9,7 +9,7 @@
 // shared memory.
 //   * A score is appended only if its order key u passes the row's threshold:
 //     u > tau, or u == tau with a key index <= tau_idx.
-//   * Every CHECK_TILES tiles, a buffer close to full is shrunk: 128 sampled
+//   * Every CHECK_TILES (2) tiles, a buffer close to full is shrunk: 128 sampled
 //     entries are ranked by comparison, and one counting pass over the buffer
 //     finds the highest of 8 sample pivots with at least k entries at or
 //     above it. Entries below that pivot are beaten by k others and are
@@ -66,7 +66,7 @@ struct IndexerTopkTile {
   static constexpr uint32_t SBO = 8 * DI;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int CAP = 4352;              // candidates per row
-  static constexpr int CHECK_TILES = 4;         // buffers are checked every 4 tiles
+  static constexpr int CHECK_TILES = 2;         // buffers are checked every 2 tiles
   static constexpr int HEADROOM = CHECK_TILES * M;
   static constexpr int MAX_K = 2048;
   static_assert(QPW * GROUPS == QG, "one row per warp group");
