@@ -3,10 +3,13 @@
 // in Top-k(I_{t,:})}); latent row = 512 value dims + 64 RoPE dims, page
 // "DeepSeek architecture", section 1.1).
 //
-// One CTA handles one query row (all H heads as the M = 128 rows of the MMA),
-// one range of selection slots (split-K for short query counts) and one slice
-// of the value dims (VSPLIT slices: an fp32 O of 128 x 512 would fill all of
-// TMEM, so the 576/512 shape runs two CTAs per row, each with a 128 x 256 O).
+// This file holds the attention parameters shared by both attention kernels,
+// the split-K combine, and the general kernel used for the small shape
+// (64-d latent, 8 heads): the 576/512 latent runs sparse_attn_vh_kernel.
+//
+// One CTA handles one query row (all H heads as the M = 128 rows of the MMA,
+// zero-padded), one range of selection slots (split-K for short query
+// counts) and one slice of the value dims (VSPLIT slices).
 //
 //   producer warps 0-3  cp.async-gather the selected latent rows (16-byte
 //                       chunks, zero-fill for empty slots) into a 128B-swizzled
