@@ -193,14 +193,23 @@ __global__ void __launch_bounds__(IndexerTile<HI, DI, QG>::THREADS, 1)
 #pragma unroll
       for (int j = 0; j < HI; ++j) cf[q][j] = coef[(qhalf * T::QPW + q) * HI + j];
 
+    // The key scale of tile i + 1 is loaded while tile i is processed, so its
+    // global-memory latency is not on the per-tile path.
+    const float* ks_row = p.k_scale + static_cast<size_t>(b) * p.n_kv;
+    auto load_ks = [&](int i) -> float {
+      const int s = (t_begin + i) * T::M + key_local;
+      return (i < n_compute && s < p.n_kv) ? ks_row[s] : 0.f;
+    };
+    float ks_next = load_ks(0);
     bool ok = true;
     for (int i = 0; i < n_compute; ++i) {
       const int buf = i & 1;
+      const float ks = ks_next;
+      ks_next = load_ks(i + 1);
       ok = mbar_wait(&acc_full[buf], (i >> 1) & 1);
       if (!ok) break;
       tc_fence_after();
       const int s = (t_begin + i) * T::M + key_local;
-      const float ks = s < p.n_kv ? p.k_scale[static_cast<size_t>(b) * p.n_kv + s] : 0.f;
 #pragma unroll
       for (int q = 0; q < T::QPW; ++q) {
         const int ql = qhalf * T::QPW + q;

@@ -570,13 +570,22 @@ __global__ void __launch_bounds__(IndexerTopkTile<HI, DI, QG>::THREADS, 1)
     // ok turns false when a bounded wait runs out (the error word is set then).
     // The loop still runs to the end, without waiting, appending or writing,
     // so that the group's barriers stay matched.
+    // The key scale of tile i + 1 is loaded while tile i is processed, so its
+    // global-memory latency is not on the per-tile path.
+    const float* ks_row = p.k_scale + static_cast<size_t>(b) * p.n_kv;
+    auto load_ks = [&](int i) -> float {
+      const int s = i * T::M + key_local;
+      return (i < n_compute && s < p.n_kv) ? ks_row[s] : 0.f;
+    };
+    float ks_next = load_ks(0);
     bool ok = true;
     for (int i = 0; i < n_compute; ++i) {
       const int buf = i & 1;
+      const float ks = ks_next;
+      ks_next = load_ks(i + 1);
       if (ok) ok = mbar_wait(&acc_full[buf], (i >> 1) & 1);
       tc_fence_after();
       const int s = i * T::M + key_local;
-      const float ks = s < p.n_kv ? p.k_scale[static_cast<size_t>(b) * p.n_kv + s] : 0.f;
       uint32_t x[T::QPW][HI];
       {
         const uint32_t col = tmem_base + lane_addr + buf * T::N + qhalf * T::QPW * HI;
