@@ -206,10 +206,18 @@ dsa_status dsa_sparse_attn_noalloc(const dsa_shape* shape, const uint16_t* q,
                                    void* stream);
 
 /*
- * The whole path for all n_q rows: indexer -> top-k -> sparse attention.
+ * The whole path for all n_q rows: indexer -> top-k -> sparse attention
+ * (page "DeepseekV3.2 拆解", eq. I_{t,s} and eq. u_t).
  *   Indexer inputs as dsa_indexer_scores, attention inputs as
  *   dsa_sparse_attn. indices_out [B, n_q, topk] receives the selection
- *   (required). Workspace: dsa_workspace_size(shape, DSA_OP_FORWARD).
+ *   (required). Workspace: dsa_workspace_size(shape, DSA_OP_FORWARD) bytes,
+ *   256-byte aligned; ws may be NULL when that is 0.
+ *   Plan: when dsa_indexer_topk supports the shape and there are at least
+ *   as many 4-row query groups as SMs (prefill), the indexer and the top-k
+ *   are one launch and no score is stored (workspace: only the attention's
+ *   split-K partials, usually none). Otherwise (decode, other shapes) the
+ *   score kernel and dsa_topk run per chunk of dsa_forward_chunk_rows()
+ *   rows, through a score buffer in the workspace.
  */
 dsa_status dsa_forward(const dsa_shape* shape, const uint8_t* q_fp8,
                        const float* q_scale, const float* w,
@@ -219,11 +227,13 @@ dsa_status dsa_forward(const dsa_shape* shape, const uint8_t* q_fp8,
                        int32_t* indices_out, void* out, int32_t out_dtype,
                        float* lse, void* ws, size_t ws_bytes, void* stream);
 
-/* Rows per indexer/top-k chunk that dsa_forward uses for this shape: the
- * scores of `rows` query rows (rows * n_kv fp32 per sequence) are the only
- * score storage, so the L x L matrix is never held at once. A caller that
- * composes the path from the stage calls gets the same launches by scoring
- * [r, r + rows) with DSA_SCORES_VISIBLE_ONLY and selecting from it. */
+/* Rows per indexer/top-k step that dsa_forward uses for this shape. With
+ * the fused plan it is n_q (one dsa_indexer_topk launch over all rows, no
+ * score storage). Otherwise the scores of `rows` query rows (rows * n_kv
+ * fp32 per sequence) are the only score storage, so the L x L matrix is
+ * never held at once; a caller that composes the path from the stage calls
+ * gets the same launches by scoring [r, r + rows) with
+ * DSA_SCORES_VISIBLE_ONLY and selecting from it. */
 dsa_status dsa_forward_chunk_rows(const dsa_shape* shape, int32_t* rows);
 
 /* Workspace bytes an op needs for this shape (0 if none). Returns status. */
