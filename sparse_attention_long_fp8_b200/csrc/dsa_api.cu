@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstdarg>
@@ -56,15 +57,16 @@ dsa_status current_device(int* dev) {
   cudaError_t e = cudaGetDevice(dev);
   if (e != cudaSuccess) return fail(DSA_ERR_NO_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
   if (*dev < 0 || *dev >= kMaxDevices) return fail(DSA_ERR_NO_DEVICE, "device ordinal out of range");
-  static int major[kMaxDevices] = {0};
-  if (major[*dev] == 0) {
-    int mj = 0;
+  // Cached per device; host threads may race to fill it, with equal values.
+  static std::atomic<int> major[kMaxDevices];
+  int mj = major[*dev].load(std::memory_order_relaxed);
+  if (mj == 0) {
     cudaDeviceGetAttribute(&mj, cudaDevAttrComputeCapabilityMajor, *dev);
-    major[*dev] = mj;
+    major[*dev].store(mj, std::memory_order_relaxed);
   }
-  if (major[*dev] != 10)
+  if (mj != 10)
     return fail(DSA_ERR_NO_DEVICE, "device %d is sm_%d0, this library is built for sm_100a", *dev,
-                major[*dev]);
+                mj);
   return DSA_OK;
 }
 
@@ -160,11 +162,13 @@ dsa_status check_attn_shape(const dsa_shape* s) {
 // ------------------------------------------------------------------ kernel attributes
 
 template <class K>
-dsa_status set_smem(K kernel, int bytes, int dev, bool* done_flags) {
-  if (!done_flags[dev]) {
+dsa_status set_smem(K kernel, int bytes, int dev, std::atomic<bool>* done_flags) {
+  // Once per device and kernel; concurrent first calls both set the same
+  // attribute, which is harmless.
+  if (!done_flags[dev].load(std::memory_order_acquire)) {
     DSA_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
                  "cudaFuncSetAttribute");
-    done_flags[dev] = true;
+    done_flags[dev].store(true, std::memory_order_release);
   }
   return DSA_OK;
 }
@@ -178,7 +182,7 @@ dsa_status launch_indexer_t(const dsa_shape* s, const uint8_t* q_fp8, const floa
                             int32_t rows, float* scores, int write_invalid, cudaStream_t stream,
                             int dev) {
   using T = dsa::IndexerTile<HI, DI, QG>;
-  static bool attr_done[kMaxDevices] = {false};
+  static std::atomic<bool> attr_done[kMaxDevices];
   if (dsa_status st = set_smem(dsa::indexer_scores_kernel<HI, DI, QG>, T::SMEM_BYTES, dev, attr_done))
     return st;
   CUtensorMap tq, tk;
@@ -246,7 +250,7 @@ dsa_status launch_indexer_topk(const dsa_shape* s, const uint8_t* q_fp8, const f
                                int32_t rows, int32_t* indices, int32_t out_rows,
                                cudaStream_t stream, int dev) {
   using T = dsa::IndexerTopkTile<64, 128, 4>;
-  static bool attr_done[kMaxDevices] = {false};
+  static std::atomic<bool> attr_done[kMaxDevices];
   if (dsa_status st = set_smem(dsa::indexer_topk_kernel<64, 128, 4>, T::SMEM_BYTES, dev, attr_done))
     return st;
   if (rows <= 0) return DSA_OK;
@@ -282,7 +286,7 @@ dsa_status launch_indexer_topk(const dsa_shape* s, const uint8_t* q_fp8, const f
 dsa_status launch_topk(const dsa_shape* s, const float* scores, int32_t row_begin, int32_t rows,
                        const int32_t* q_pos0, const int32_t* kv_len, int32_t* indices,
                        int32_t out_rows, int32_t out_row0, cudaStream_t stream, int dev) {
-  static bool attr_done[kMaxDevices] = {false};
+  static std::atomic<bool> attr_done[kMaxDevices];
   const int smem = static_cast<int>(sizeof(dsa::TopkSmem));
   if (dsa_status st = set_smem(dsa::topk_kernel, smem, dev, attr_done)) return st;
   if (s->batch > 65535) return fail(DSA_ERR_INVALID_ARG, "batch > 65535");
@@ -340,7 +344,7 @@ dsa_status launch_attn_t(const dsa_shape* s, const AttnPlan& pl, const uint16_t*
                          const uint16_t* kv, const int32_t* indices, void* out, int out_bf16,
                          float* lse, void* ws, cudaStream_t stream, int dev) {
   using T = dsa::AttnTile<DQK, DV, VSPLIT>;
-  static bool attr_done[kMaxDevices] = {false};
+  static std::atomic<bool> attr_done[kMaxDevices];
   if (dsa_status st = set_smem(dsa::sparse_attn_kernel<DQK, DV, VSPLIT>, T::SMEM_BYTES, dev, attr_done))
     return st;
   dsa::AttnParams p{};
@@ -383,7 +387,7 @@ dsa_status launch_attn_vh(const dsa_shape* s, const AttnPlan& pl, const uint16_t
                             const uint16_t* kv, const int32_t* indices, void* out, int out_bf16,
                             float* lse, void* ws, cudaStream_t stream, int dev) {
   using T = dsa::VhTile;
-  static bool attr_done[kMaxDevices] = {false};
+  static std::atomic<bool> attr_done[kMaxDevices];
   if (dsa_status st = set_smem(dsa::sparse_attn_vh_kernel, T::SMEM_BYTES, dev, attr_done))
     return st;
   dsa::AttnParams p{};
