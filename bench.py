@@ -3,14 +3,17 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-A step is one pass of the whole path over one batch of synthetic input: the
-lightning indexer with its top-k selection (one fused kernel for prefill; a
-score kernel and a selection kernel per row chunk for decode), then the
-sparse attention over all rows, composed from the library's stage calls
-exactly as dsa_forward launches them, so each kernel can be timed with CUDA
-events on its stream. The headline workload is DSA prefill at L = 65536 (batch 1,
-H^I = 64, d^I = 128, k = 2048, 128-head MQA over the 576-d latent); batch
-decode (64 x 32768 and 64 x 65536 cached tokens) is measured after it.
+A step is one call of the public ``dsa_forward`` over one batch of synthetic
+input: the lightning indexer with its top-k selection (one fused kernel for
+prefill; a score kernel and a selection kernel per row chunk for decode),
+then the sparse attention over all rows. The headline workload is DSA
+prefill at L = 65536 (batch 1, H^I = 64, d^I = 128, k = 2048, 128-head MQA
+over the 576-d latent); prefill at L = 16384 and batch decode (64 x 32768
+and 64 x 65536 cached tokens) are measured after it.
+
+The step time is K timed dsa_forward calls between CUDA events. A second,
+eager pass runs the same launches through the library's stage calls with
+events around each kernel: it gives the per-kernel times the rooflines use.
 
 Rank 0 prints ONE JSON line on stdout; everything else goes to stderr.
 Under torchrun every rank runs its own independent problem (weak scaling,
@@ -81,20 +84,21 @@ def attn_flops(cfg):
 
 
 def decode_bytes(cfg):
-    """Algorithmic HBM bytes of one decode step (each byte the path must move
-    once): indexer key cache (fp8 + scale), query-side indexer inputs, the
-    fp32 score row written and read once by top-k, the selected indices, the
-    gathered latent rows, q, and the fp32 output."""
+    """Algorithmic HBM bytes of one decode step, the bytes the path must move
+    once: the indexer key cache (fp8 codes + scale), the query-side indexer
+    inputs (codes, scale, weight), the selected indices, the gathered latent
+    rows, bf16 q, and the fp32 output with its LSE. Scores are not counted:
+    storing them is a choice of the implementation, not part of the path."""
     B, S, k = cfg.batch, cfg.n_kv, min(cfg.topk, cfg.n_kv)
     kcache = B * S * (cfg.idx_dim + 4)
     qside = B * cfg.idx_heads * (cfg.idx_dim + 8)
-    scores = 2 * B * S * 4
-    idx = 2 * B * k * 4
+    idx = B * k * 4
     gather = B * k * cfg.qk_dim * 2
     q = B * cfg.heads * cfg.qk_dim * 2
     out = B * cfg.heads * (cfg.v_dim * 4 + 4)
-    return {"total": kcache + qside + scores + idx + gather + q + out,
-            "attention": gather + q + out + B * k * 4}
+    return {"total": kcache + qside + idx + gather + q + out,
+            "attention": gather + q + out + idx,
+            "indexer": kcache + qside}
 
 
 # ---------------------------------------------------------------- clocks
@@ -163,7 +167,9 @@ def measured_peaks():
 # ---------------------------------------------------------------- the step
 
 class Step:
-    """The path for one workload, composed from the library's stage calls."""
+    """The path for one workload: the public dsa_forward call (the timed
+    step) and the same launches through the stage calls (the per-kernel
+    breakdown), following the plan dsa_forward_plan reports."""
 
     def __init__(self, cfg, seed, device):
         import torch
@@ -172,9 +178,11 @@ class Step:
         self.inp = dsa.make_inputs(cfg, seed=seed, device=device)
         self.shape = dsa.shape_of(cfg)
         B, T = cfg.batch, cfg.n_q
-        self.chunk = dsa.forward_chunk_rows(self.shape)
+        plan = dsa.forward_plan(self.shape)
+        self.fused, self.chunk = plan["fused"], plan["chunk_rows"]
+        self.attn_splits = plan["attn_splits"]
         self.attn_ws_bytes = dsa.workspace_size(self.shape, dsa.DSA_OP_SPARSE_ATTN)
-        self.fwd_ws_bytes = dsa.workspace_size(self.shape, dsa.DSA_OP_FORWARD)
+        self.fwd_ws, self.fwd_ws_bytes = dsa.alloc_workspace(self.shape, dsa.DSA_OP_FORWARD, device)
         self.attn_ws = torch.empty(max(self.attn_ws_bytes, 256), dtype=torch.uint8, device=device)
         self.idx = torch.empty(B, T, cfg.topk, dtype=torch.int32, device=device)
         self.out = torch.empty(B, T, cfg.heads, cfg.v_dim, device=device)
@@ -182,17 +190,22 @@ class Step:
         self.chunks = [(r0, min(T, r0 + self.chunk)) for r0 in range(0, T, self.chunk)]
         if B > 1 and len(self.chunks) > 1:
             raise ValueError("stage composition needs one chunk when batch > 1")
-        # dsa_forward's plan: the fused indexer + selection needs no score
-        # buffer, so its forward workspace is the attention's alone.
-        self.fused = self.fwd_ws_bytes == self.attn_ws_bytes
         self.scores = None if self.fused else torch.empty(B, min(self.chunk, T), cfg.n_kv,
                                                           device=device)
         per_chunk = 1 if self.fused else 2
-        self.launches = per_chunk * len(self.chunks) + 1 + (1 if self.attn_ws_bytes > 0 else 0)
+        self.launches = per_chunk * len(self.chunks) + 1 + (1 if self.attn_splits > 1 else 0)
+
+    def run_forward(self):
+        """One step through the public call."""
+        x = self.inp
+        self.dsa.dsa_forward(self.shape, x["q_fp8"], x["q_scale"], x["w"], x["k_fp8"],
+                             x["k_scale"], x["q_pos0"], x["kv_len"], x["q"], x["kv"], self.idx,
+                             self.out, self.lse, self.fwd_ws, self.fwd_ws_bytes)
 
     def run(self, ev=None):
-        """One step; with ev = (list of (start, end) event pairs per stage) the
-        stage boundaries are recorded on the current stream."""
+        """The same launches through the stage calls; with ev (a dict of event
+        lists per stage) each launch is bracketed by events on the current
+        stream."""
         dsa, x, cfg = self.dsa, self.inp, self.cfg
         rec = (lambda name: ev[name].append(self.torch.cuda.Event(enable_timing=True)) or
                ev[name][-1].record()) if ev is not None else (lambda name: None)
@@ -287,27 +300,23 @@ def stage_ms(ev):
 
 
 def timed(step, steps, warmup, dist, graph=False):
-    """W untimed steps, then K timed steps between barriers; returns
-    (ms per step as max over ranks, per-stage event timings).
+    """W untimed steps, then K timed dsa_forward calls between barriers and
+    CUDA events; returns ms per step as the max over ranks.
 
     With graph=True (short, launch-bound steps: decode) the step is captured
-    once into a CUDA graph and the K timed steps are graph replays; the
-    per-stage times then come from a separate eager pass with events."""
+    once into a CUDA graph and the K timed steps are graph replays."""
     import torch
     for _ in range(warmup):
-        step.run()
+        step.run_forward()
     torch.cuda.synchronize()
     step.dsa.dsa_check()
-    ev = {"indexer": [], "topk": [], "attn": []}
     g = None
     if graph:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            step.run()
+            step.run_forward()
         for _ in range(warmup):
             g.replay()
-        for _ in range(steps):      # the eager pass for the stage breakdown
-            step.run(ev)
         torch.cuda.synchronize()
         step.dsa.dsa_check()
     if dist:
@@ -319,7 +328,7 @@ def timed(step, steps, warmup, dist, graph=False):
         if g is not None:
             g.replay()
         else:
-            step.run(ev)
+            step.run_forward()
     end.record()
     torch.cuda.synchronize()
     if dist:
@@ -327,7 +336,98 @@ def timed(step, steps, warmup, dist, graph=False):
     step.dsa.dsa_check()
     ms = max_over_ranks(start.elapsed_time(end) / steps, dist)
     del g
-    return ms, stage_ms(ev)
+    return ms
+
+
+def breakdown(step, steps):
+    """K eager steps through the stage calls, each launch between CUDA events
+    on the launching stream: per-kernel times for the rooflines."""
+    import torch
+    ev = {"indexer": [], "topk": [], "attn": []}
+    step.run()
+    torch.cuda.synchronize()
+    for _ in range(steps):
+        step.run(ev)
+    torch.cuda.synchronize()
+    step.dsa.dsa_check()
+    return stage_ms(ev)
+
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# sparse_attn_vh_kernel over the 4096-row prefill, from one ncu capture, and
+# the SHA-256 of the kernel source that capture ran. The kernel's traffic is
+# q read once plus out and lse written once (the latent gathers hit L2), so it
+# grows in proportion to the rows and is scaled by them. When the source no
+# longer matches, the figure is stale and the line reports null.
+ATTN_TRAFFIC_4K = {"bytes": 642.484736e6 + 1022.602e6, "rows": 4096,
+                   "source_sha256": "fc29016b7b6d77133fd629c9c6d3f7a7b7751e164c765ab4709e0c1e29010395"}
+
+
+def kernel_source_sha256(name):
+    import hashlib
+    path = os.path.join(ROOT, "sparse_attention_long_fp8_b200", "csrc", name)
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()
+
+
+def attn_traffic(cfg):
+    """Per-launch DRAM bytes of the attention kernel at cfg, or None when the
+    captured figure does not belong to the current kernel source."""
+    cap = ATTN_TRAFFIC_4K
+    if cap["source_sha256"] != kernel_source_sha256("sparse_attn_vh.cuh"):
+        return None
+    return cap["bytes"] / cap["rows"] * cfg.batch * cfg.n_q
+
+
+def prefill_leg(cfg, seed, steps, warmup, dist, peaks):
+    """dsa_forward over one prefill workload: tokens/s from the timed calls,
+    per-kernel TFLOP/s from the breakdown pass."""
+    import torch
+    step = Step(cfg, seed, "cuda")
+    log(f"[bench] {cfg.name}: fused {step.fused}, chunk rows {step.chunk}, "
+        f"{step.launches} launches/step")
+    ms = timed(step, steps, warmup, dist)
+    stages = breakdown(step, steps)
+    launches = step.launches
+    fused = step.fused
+    del step
+    torch.cuda.empty_cache()
+    per = {k: v["total_ms"] / steps for k, v in stages.items()}
+    ix_f, at_f = indexer_flops(cfg), attn_flops(cfg)
+    fp8_peak = 2.0 * peaks["bf16_sustained"]
+    ix_ms = per["indexer"] + (0.0 if fused else per["topk"])
+    res = {"ms_per_step": ms, "tokens_per_s": cfg.batch * cfg.n_q / (ms / 1e3),
+           "stages_ms": ({"indexer_topk_fused": per["indexer"], "attention": per["attn"]}
+                         if fused else {"indexer": per["indexer"], "topk": per["topk"],
+                                        "attention": per["attn"]}),
+           "stage_sum_ms": sum(per.values()),
+           "indexer_tflops_fp8": ix_f / (ix_ms / 1e3) / 1e12,
+           "attention_tflops_bf16": at_f / (per["attn"] / 1e3) / 1e12,
+           "launches_per_step": launches}
+    res["indexer_frac_fp8"] = res["indexer_tflops_fp8"] / fp8_peak
+    res["attention_frac_bf16"] = res["attention_tflops_bf16"] / peaks["bf16_sustained"]
+    return res, stages, fused
+
+
+def decode_leg(cfg, seed, steps, warmup, dist, peaks):
+    """Batch decode: dsa_forward captured in a CUDA graph (a step is ~0.2 ms
+    of a few launches), bytes per step as decode_bytes counts them."""
+    import torch
+    step = Step(cfg, seed, "cuda")
+    ms = timed(step, steps, warmup, dist, graph=True)
+    stages = breakdown(step, steps)
+    launches = step.launches
+    del step
+    torch.cuda.empty_cache()
+    nb = decode_bytes(cfg)
+    per = {k: v["total_ms"] / steps for k, v in stages.items()}
+    gbs = nb["total"] / (ms / 1e3) / 1e9
+    return {"ms_per_step": ms, "GB_per_s": gbs, "frac_hbm": gbs / peaks["hbm"],
+            "attention_ms": per["attn"],
+            "attention_GB_per_s": nb["attention"] / (per["attn"] / 1e3) / 1e9,
+            "indexer_GB_per_s": nb["indexer"] / (per["indexer"] / 1e3) / 1e9,
+            "stages_ms": per, "launches_per_step": launches,
+            "timing": "CUDA graph replays of dsa_forward; stages from an eager pass",
+            "algorithmic_bytes": nb["total"]}
 
 
 # ---------------------------------------------------------------- e2e
@@ -406,26 +506,38 @@ def host_available_bytes():
 
 # ---------------------------------------------------------------- CPU oracle
 
-def oracle_rows_per_s(cfg, seed, n_rows):
-    """The fp64 oracle (as it stands) over n_rows evenly spaced query rows of
-    the workload on this host's cores; evenly spaced rows have the workload's
-    average per-row cost, so rows/s extrapolates to the whole config."""
+def oracle_sample_rows(cfg, n_rows, offset=0.5):
+    """n_rows evenly spaced query rows of the workload (offset in [0, 1)
+    shifts them within their spacing); evenly spaced rows have the
+    workload's average per-row cost, so rows/s extrapolates to the whole
+    config."""
+    import numpy as np
+    T = cfg.n_q
+    return np.unique(((np.arange(n_rows) + offset) * T / n_rows).astype(np.int64))
+
+
+def oracle_inputs(cfg, seed):
+    """The workload's inputs, drawn once (on the GPU when there is one: the
+    drawing is not timed)."""
+    import torch
+    from sparse_attention_long_fp8_b200 import inputs
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    return inputs.make_inputs(cfg, seed=seed, device=dev)
+
+
+def oracle_rows_per_s(cfg, inp, rows):
+    """The fp64 oracle (as it stands) over the given query rows of sequence
+    0 on this host's cores: (rows/s, seconds, threads used, rows)."""
     import numpy as np
     import torch
     import oracle
-    from sparse_attention_long_fp8_b200 import inputs
-    dev = "cuda" if torch.cuda.is_available() else "cpu"
-    inp = inputs.make_inputs(cfg, seed=seed, device=dev)
-    T = cfg.n_q
-    rows = np.unique(((np.arange(n_rows) + 0.5) * T / n_rows).astype(np.int64))
     sel = torch.as_tensor(rows, device=inp["q_fp8"].device)
     small = {"q_fp8": inp["q_fp8"][:, sel].cpu(), "q_scale": inp["q_scale"][:, sel].cpu(),
              "w": inp["w"][:, sel].cpu(), "k_fp8": inp["k_fp8"].cpu(),
              "k_scale": inp["k_scale"].cpu(), "q": inp["q"][:, sel].cpu(),
              "kv": inp["kv"].cpu(), "q_pos0": inp["q_pos0"].cpu(), "kv_len": inp["kv_len"].cpu()}
-    del inp
     b = 0
-    pos = (rows + int(small["q_pos0"][b])).astype(np.int32)
+    pos = (np.asarray(rows) + int(small["q_pos0"][b])).astype(np.int32)
     t0 = time.perf_counter()
     sc = oracle.indexer_scores(small["q_fp8"][b], small["q_scale"][b], small["w"][b],
                                small["k_fp8"][b], small["k_scale"][b], pos,
@@ -464,41 +576,30 @@ def main():
     seed = 1000 + rank
 
     clocks = ClockSampler(local)
-    step = Step(cfg, seed, "cuda")
-    log(f"[bench] {cfg.name}: chunk rows {step.chunk}, {len(step.chunks)} chunks, "
-        f"{step.launches} launches/step")
     clocks.start()
-    ms, stages = timed(step, args.steps, args.warmup, dist)
+    head, stages, fused = prefill_leg(cfg, seed, args.steps, args.warmup, dist, peaks)
     clock_info = clocks.stop()
-    fused = step.fused
-    del step
-    torch.cuda.empty_cache()
-
+    ms = head["ms_per_step"]
     tokens = cfg.batch * cfg.n_q
     value = world * tokens / (ms / 1e3)
-    ix_f, at_f = indexer_flops(cfg), attn_flops(cfg)
-    ix_ms = stages["indexer"]["total_ms"] / args.steps
-    at_ms = stages["attn"]["total_ms"] / args.steps
-    tk_ms = stages["topk"]["total_ms"] / args.steps
-    fp8_peak = 2.0 * peaks["bf16_sustained"]
-    ix_tf = ix_f / (ix_ms / 1e3) / 1e12
-    at_tf = at_f / (at_ms / 1e3) / 1e12
-    dominant = max(("indexer", ix_ms), ("attn", at_ms), ("topk", tk_ms), key=lambda x: x[1])[0]
-    ix_kernel = "indexer_topk_kernel<64,128,4>" if fused else "indexer_scores_kernel<64,128,4>"
+
+    per = {k: v["total_ms"] / args.steps for k, v in stages.items()}
+    at_ms, ix_ms = per["attn"], per["indexer"]
+    dominant = max(("indexer", ix_ms), ("attn", at_ms), ("topk", per["topk"]),
+                   key=lambda x: x[1])[0]
     if dominant == "attn":
-        # DRAM bytes of sparse_attn_vh_kernel from one ncu capture at L = 4096
-        # (dram__bytes_read.sum + dram__bytes_write.sum = 642.5 MB + 1022.6 MB,
-        # profiles/ncu_full_prefill_4k.md); its traffic grows in proportion to
-        # the query rows, so it is scaled by rows. Re-capture when the kernel
-        # changes.
-        traffic = (642.484736e6 + 1022.602e6) / 4096 * cfg.batch * cfg.n_q
+        traffic = attn_traffic(cfg)
         roof = {"kernel": "sparse_attn_vh_kernel", "bound": "tensor",
-                "achieved": at_f / (at_ms / 1e3) / 1e12, "peak": peaks["bf16_sustained"],
+                "achieved": head["attention_tflops_bf16"], "peak": peaks["bf16_sustained"],
                 "unit": "TFLOP/s", "traffic": traffic,
-                "traffic_source": "ncu DRAM bytes of one 4096-row launch, scaled by rows"}
+                "traffic_source": ("ncu DRAM bytes of one 4096-row launch of the same kernel "
+                                   "source, scaled by rows") if traffic else
+                                  "null: no capture of the current kernel source"}
     elif dominant == "indexer":
-        roof = {"kernel": ix_kernel, "bound": "tensor",
-                "achieved": ix_tf, "peak": fp8_peak, "unit": "TFLOP/s", "traffic": None}
+        kern = "indexer_topk_kernel<64,128,4>" if fused else "indexer_scores_kernel<64,128,4>"
+        roof = {"kernel": kern, "bound": "tensor",
+                "achieved": indexer_flops(cfg) / (ix_ms / 1e3) / 1e12,
+                "peak": 2.0 * peaks["bf16_sustained"], "unit": "TFLOP/s", "traffic": None}
     else:
         roof = {"kernel": "topk_kernel", "bound": "hbm", "achieved": None,
                 "peak": peaks["hbm"], "unit": "GB/s", "traffic": None}
@@ -506,6 +607,7 @@ def main():
         roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = f"{peaks['source']} ({'bf16 sustained' if roof['unit'] == 'TFLOP/s' else 'hbm copy'}" + \
         (", x2 for fp8" if roof.get("kernel", "").startswith("indexer") else "") + ")"
+    roof["launches_timed"] = stages[dominant]["launches"]
 
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -514,37 +616,26 @@ def main():
         "dtype": "fp8e4m3 indexer, bf16 attention, fp32 accumulate",
         "data": "synthetic (seeded; page-shaped workloads)",
         "config": bench_config(cfg, world),
-        "stages_ms": ({"indexer_topk_fused": ix_ms, "attention": at_ms} if fused else
-                      {"indexer": ix_ms, "topk": tk_ms, "attention": at_ms}),
-        "indexer_tflops_fp8": ix_tf, "indexer_frac_fp8": ix_tf / fp8_peak,
-        "attention_tflops_bf16": at_tf, "attention_frac_bf16": at_tf / peaks["bf16_sustained"],
-        "roofline": roof, "gpu_launches": step_launches_total(stages),
+        "stages_ms": head["stages_ms"], "stage_sum_ms": head["stage_sum_ms"],
+        "indexer_tflops_fp8": head["indexer_tflops_fp8"],
+        "indexer_frac_fp8": head["indexer_frac_fp8"],
+        "attention_tflops_bf16": head["attention_tflops_bf16"],
+        "attention_frac_bf16": head["attention_frac_bf16"],
+        "roofline": roof, "gpu_launches": head["launches_per_step"] * args.steps,
         "clocks": clock_info,
     }
 
-    if not args.no_decode:
+    if not args.no_decode and args.workload == HEADLINE:
+        pcfg = inputs.CONFIGS["prefill_16k"]
+        leg, _, _ = prefill_leg(pcfg, seed, args.steps, args.warmup, dist, peaks)
+        result["prefill_16k"] = leg
         result["quantiser"] = quantiser_bench(cfg, peaks)
-
-    if not args.no_decode:
         result["decode"] = {}
         for name in ("decode_32k", "decode_64k"):
-            dcfg = inputs.CONFIGS[name]
-            dstep = Step(dcfg, seed, "cuda")
-            # decode steps are ~0.2 ms: many of them, after a longer warm-up,
-            # replayed from a CUDA graph
-            dsteps = max(args.steps, 100)
-            dms, dst = timed(dstep, dsteps, max(args.warmup, 20), dist, graph=True)
-            nb = decode_bytes(dcfg)
-            at = dst["attn"]["total_ms"] / dsteps
-            result["decode"][name] = {
-                "ms_per_step": dms, "GB_per_s": nb["total"] / (dms / 1e3) / 1e9,
-                "frac_hbm": nb["total"] / (dms / 1e3) / 1e9 / peaks["hbm"],
-                "attention_ms": at,
-                "attention_GB_per_s": nb["attention"] / (at / 1e3) / 1e9,
-                "stages_ms": {k: v["total_ms"] / dsteps for k, v in dst.items()},
-                "timing": "CUDA graph replays of the step; stages from an eager pass",
-                "algorithmic_bytes": nb["total"]}
-            del dstep
+            # decode steps are ~0.2 ms: many of them, after a longer warm-up
+            result["decode"][name] = decode_leg(inputs.CONFIGS[name], seed,
+                                                max(args.steps, 100), max(args.warmup, 20),
+                                                dist, peaks)
             torch.cuda.empty_cache()
 
     # The ranks of a node share its host RAM: every rank needs its own pinned
@@ -566,13 +657,15 @@ def main():
 
     if not args.no_cpu and world == 1 and rank == 0:
         # A calibration sample of one row per host thread, then a sample
-        # sized for about 12 s of oracle work.
+        # sized for about 12 s of oracle work, on every host thread.
         import oracle
         threads = max(1, oracle.hardware_threads())
-        _, dt0, _, nr0 = oracle_rows_per_s(cfg, seed, threads)
+        oinp = oracle_inputs(cfg, seed)
+        _, dt0, _, nr0 = oracle_rows_per_s(cfg, oinp, oracle_sample_rows(cfg, threads))
         reps = max(1, min(32, int(12.0 / max(dt0, 1e-3))))
         n_rows = min(cfg.n_q, nr0 * reps)
-        rps, dt, cores, nr = oracle_rows_per_s(cfg, seed, n_rows)
+        rps, dt, cores, nr = oracle_rows_per_s(cfg, oinp, oracle_sample_rows(cfg, n_rows))
+        del oinp
         result["cpu_baseline"] = {"value": rps * cfg.batch, "unit": "tokens/s", "cores": cores,
                                   "kind": "oracle",
                                   "sample": f"{nr} evenly spaced query rows of {cfg.name} "
@@ -594,27 +687,29 @@ def bench_config(cfg, world):
             "l2": "inputs larger than L2 (q is 9.7 GB per step)"}
 
 
-def step_launches_total(stages):
-    return sum(v["launches"] for v in stages.values())
-
-
 def main_reference(args, world, rank):
     """The reference arm: the fp64 oracle as it stands on this host's cores,
     same workload, metric and unit; each step is a bounded sample of rows."""
     if rank != 0:
         return
     from sparse_attention_long_fp8_b200 import inputs
+    import oracle
     cfg = inputs.CONFIGS[args.workload]
-    n_rows = 8
-    for _ in range(args.warmup):
-        oracle_rows_per_s(cfg, 7, 2)
-    rates, secs, cores = [], [], 1
-    for i in range(args.steps):
-        rps, dt, cores, nr = oracle_rows_per_s(cfg, 1000 + i, n_rows)
-        rates.append(rps)
-        secs.append(dt)
-    value = len(rates) * n_rows / sum(secs)
-    sample = f"{n_rows} evenly spaced query rows of {cfg.name} per step (fp64 oracle)"
+    # One sampled row per host thread and step, so every thread works; the
+    # steps take differently offset evenly spaced rows of one drawn input.
+    n_rows = min(cfg.n_q, max(1, oracle.hardware_threads()))
+    inp = oracle_inputs(cfg, 1000)
+    total = args.warmup + args.steps
+    secs, cores, done = [], 1, 0
+    for i in range(total):
+        rows = oracle_sample_rows(cfg, n_rows, offset=(i + 0.5) / total)
+        _, dt, cores, nr = oracle_rows_per_s(cfg, inp, rows)
+        if i >= args.warmup:
+            secs.append(dt)
+            done += nr
+    value = done / sum(secs)
+    sample = (f"{n_rows} evenly spaced query rows of {cfg.name} per step on {cores} threads "
+              f"(fp64 oracle: indexer + top-k + attention)")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

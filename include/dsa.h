@@ -15,8 +15,15 @@
  *
  * Conventions shared by every call
  *   - Every pointer argument is a DEVICE pointer, allocated and owned by the
- *     caller. The library allocates no device memory and keeps no pointer
- *     after a call returns.
+ *     caller. No call allocates device memory and the library keeps no
+ *     caller pointer after a call returns. The one exception to "no library
+ *     memory" is static: the 16 MiB scratch array of
+ *     dsa_sparse_attn_noalloc, which every GPU that loads the library holds
+ *     until the process exits.
+ *   - Per-device facts (kernel attributes, the SM count, the scratch array's
+ *     address) are looked up on first use and cached for the process. Do
+ *     not use the library across a cudaDeviceReset (or any teardown of the
+ *     device's primary context): the cached state would be stale.
  *   - Every call is asynchronous on the caller's CUDA stream (`stream`, a
  *     cudaStream_t passed as void*; NULL = legacy default stream). No call
  *     synchronises except dsa_check().
@@ -235,6 +242,18 @@ dsa_status dsa_forward(const dsa_shape* shape, const uint8_t* q_fp8,
  * gets the same launches by scoring [r, r + rows) with
  * DSA_SCORES_VISIBLE_ONLY and selecting from it. */
 dsa_status dsa_forward_chunk_rows(const dsa_shape* shape, int32_t* rows);
+
+/* The plan dsa_forward takes for this shape, for callers that compose the
+ * path from the stage calls (or time its kernels one by one):
+ *   *fused       1 when the indexer and the top-k run as one
+ *                dsa_indexer_topk launch over all rows, else 0 (score kernel
+ *                + dsa_topk per chunk of *chunk_rows rows);
+ *   *chunk_rows  as dsa_forward_chunk_rows;
+ *   *attn_splits split-K factor of the attention (1 = no partials, else a
+ *                combine kernel follows the attention kernel).
+ * Host-only; a shape outside the compiled set returns its error. */
+dsa_status dsa_forward_plan(const dsa_shape* shape, int32_t* fused, int32_t* chunk_rows,
+                            int32_t* attn_splits);
 
 /* Workspace bytes an op needs for this shape (0 if none). Returns status. */
 dsa_status dsa_workspace_size(const dsa_shape* shape, int32_t op,

@@ -82,13 +82,15 @@ def load_library(path: str | None = None):
     lib.dsa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P]
     lib.dsa_selftest_wait_timeout.restype = ctypes.c_int
     lib.dsa_forward_chunk_rows.argtypes = [SP, ctypes.POINTER(I32)]
+    lib.dsa_forward_plan.argtypes = [SP, ctypes.POINTER(I32), ctypes.POINTER(I32),
+                                     ctypes.POINTER(I32)]
     lib.dsa_status_string.argtypes = [ctypes.c_int]
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_last_error.restype = ctypes.c_char_p
     lib.dsa_version.restype = ctypes.c_char_p
     for fn in ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
                "dsa_workspace_size", "dsa_check", "dsa_forward_chunk_rows",
-               "dsa_sparse_attn_noalloc"):
+               "dsa_sparse_attn_noalloc", "dsa_forward_plan"):
         getattr(lib, fn).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -147,6 +149,14 @@ def forward_chunk_rows(shape: DsaShape) -> int:
     n = ctypes.c_int32(0)
     _raise(load_library().dsa_forward_chunk_rows(ctypes.byref(shape), ctypes.byref(n)))
     return n.value
+
+
+def forward_plan(shape: DsaShape) -> dict:
+    """dsa_forward's plan for this shape: fused (bool), chunk_rows, attn_splits."""
+    f, c, sp = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
+    _raise(load_library().dsa_forward_plan(ctypes.byref(shape), ctypes.byref(f), ctypes.byref(c),
+                                           ctypes.byref(sp)))
+    return {"fused": bool(f.value), "chunk_rows": c.value, "attn_splits": sp.value}
 
 
 def dsa_indexer_scores(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,

@@ -48,8 +48,30 @@ dsa_status cuda_fail(cudaError_t e, const char* what) {
     if (e_ != cudaSuccess) return cuda_fail(e_, what); \
   } while (0)
 
-constexpr int kNumSms = 148;
 constexpr int kMaxDevices = 64;
+// SM count assumed when no device is current (host-only size queries).
+constexpr int kDefaultSms = 148;
+
+// SM count of the current device, read once per device. It sizes grids and
+// decides the split plans, so dsa_workspace_size and the launches that use
+// the workspace see the same value on the same device.
+int num_sms() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();   // no device: clear the non-sticky error
+    return kDefaultSms;
+  }
+  static std::atomic<int> sms[kMaxDevices];
+  int n = sms[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = kDefaultSms;
+    }
+    sms[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
 
 // ------------------------------------------------------------------ device check
 
@@ -205,7 +227,8 @@ dsa_status launch_indexer_t(const dsa_shape* s, const uint8_t* q_fp8, const floa
   p.n_groups = (rows + QG - 1) / QG;
   const int n_tiles = (s->n_kv + T::M - 1) / T::M;
   const int64_t groups = static_cast<int64_t>(s->batch) * p.n_groups;
-  int64_t tps = (groups * n_tiles + 4 * kNumSms - 1) / (4 * kNumSms);
+  const int sms = num_sms();
+  int64_t tps = (groups * n_tiles + 4 * sms - 1) / (4 * sms);
   tps = std::max<int64_t>(4, std::min<int64_t>(tps, 64));
   tps = std::min<int64_t>(tps, n_tiles);
   p.tiles_per_split = static_cast<int32_t>(tps);
@@ -321,8 +344,9 @@ AttnPlan plan_attn(const dsa_shape* s) {
   const int64_t ctas = rows * pl.vsplit;
   const int max_splits = (s->topk + 31) / 32;
   int splits = 1;
-  if (ctas < kNumSms / 2) {
-    splits = static_cast<int>(std::min<int64_t>(max_splits, (kNumSms + ctas - 1) / ctas));
+  const int sms = num_sms();
+  if (ctas < sms / 2) {
+    splits = static_cast<int>(std::min<int64_t>(max_splits, (sms + ctas - 1) / ctas));
     splits = std::max(1, std::min(splits, 16));
   }
   int sps = (s->topk + splits - 1) / splits;
@@ -454,7 +478,7 @@ FwdPlan plan_forward(const dsa_shape* s) {
   // with fewer groups than SMs (decode) the split score kernel plus the
   // separate selection keeps more of the GPU busy.
   const int64_t groups = static_cast<int64_t>(s->batch) * ((s->n_q + 3) / 4);
-  if (indexer_topk_supported(s) && groups >= kNumSms) {
+  if (indexer_topk_supported(s) && groups >= num_sms()) {
     f.fused = true;
     f.chunk_rows = s->n_q;
     f.scores_bytes = 0;
@@ -595,6 +619,19 @@ dsa_status dsa_forward_chunk_rows(const dsa_shape* s, int32_t* rows) {
   if (dsa_status st = check_indexer_shape(s)) return st;
   if (dsa_status st = check_attn_shape(s)) return st;
   *rows = plan_forward(s).chunk_rows;
+  return DSA_OK;
+}
+
+dsa_status dsa_forward_plan(const dsa_shape* s, int32_t* fused, int32_t* chunk_rows,
+                            int32_t* attn_splits) {
+  if (!fused || !chunk_rows || !attn_splits)
+    return fail(DSA_ERR_INVALID_ARG, "dsa_forward_plan: output pointer is NULL");
+  if (dsa_status st = check_indexer_shape(s)) return st;
+  if (dsa_status st = check_attn_shape(s)) return st;
+  const FwdPlan f = plan_forward(s);
+  *fused = f.fused ? 1 : 0;
+  *chunk_rows = f.chunk_rows;
+  *attn_splits = plan_attn(s).splits;
   return DSA_OK;
 }
 

@@ -33,14 +33,23 @@ def test_headline_flop_counts():
 
 
 def test_decode_bytes_at_both_contexts():
-    """Per step: FP8 key cache + scales, query-side indexer inputs, the score
-    row written and read, the indices written and read, the gathered latent
-    rows, bf16 q and the fp32 output with its LSE."""
-    for name, S, want_mb in [("decode_32k", 32768, 472.4), ("decode_64k", 65536, 766.1)]:
+    """Per step: FP8 key cache + scales, query-side indexer inputs (codes,
+    scale, weight), the indices, the gathered latent rows, bf16 q and the
+    fp32 output with its LSE; no score round trip (the scope table's
+    ~456 MB at 32768 and ~733 MB at 65536)."""
+    for name, S, want_mb in [("decode_32k", 32768, 455.1), ("decode_64k", 65536, 731.9)]:
         cfg = inputs.CONFIGS[name]
         B, k = 64, 2048
-        total = (B * S * (128 + 4) + B * 64 * (128 + 4 + 4) + 2 * B * S * 4 + 2 * B * k * 4
+        total = (B * S * (128 + 4) + B * 64 * (128 + 4 + 4) + B * k * 4
                  + B * k * 576 * 2 + B * 128 * 576 * 2 + B * 128 * (512 * 4 + 4))
         got = bench.decode_bytes(cfg)["total"]
         assert got == total
         assert abs(got / 1e6 - want_mb) < 0.5
+
+
+def test_sampled_oracle_rows_are_evenly_spaced_and_distinct():
+    cfg = inputs.CONFIGS["prefill_64k"]
+    for n, off in [(16, 0.5), (16, 0.01), (272, 0.99), (1, 0.5)]:
+        rows = bench.oracle_sample_rows(cfg, n, off)
+        assert len(rows) == n and rows.min() >= 0 and rows.max() < cfg.n_q
+        assert (abs((rows[1:] - rows[:-1]) - cfg.n_q / n) <= 1).all()

@@ -162,10 +162,24 @@ def _fused(cfg, g, rb, re_):
 def _assert_same_sets(a, b):
     """Both kernels form each score with the same fp32 operations, so the
     selected sets must be identical (integer work: bit-exact)."""
-    a = np.sort(a.cpu().numpy(), axis=-1)
-    b = np.sort(b.cpu().numpy(), axis=-1)
+    a = np.sort(a.cpu().numpy() if torch.is_tensor(a) else np.asarray(a), axis=-1)
+    b = np.sort(b.cpu().numpy() if torch.is_tensor(b) else np.asarray(b), axis=-1)
     bad = np.nonzero((a != b).any(axis=-1))
     assert a.shape == b.shape and len(bad[0]) == 0, f"rows differ: {list(zip(*bad))[:8]}"
+
+
+def _check_fused_against_oracle(cfg, inp, g, rb, re_, fused, band_rows):
+    """The fused selection against the oracle directly:
+    * exact: the oracle's top-k (full sort, ties to the lower index) of the
+      GPU's own fp32 scores of every tested row gives the same sets;
+    * band: on sampled rows, against the oracle's fp64 scores."""
+    sc = _gpu_scores(cfg, g, rb, re_).double().cpu().numpy()
+    got = fused.cpu().numpy()
+    for b in range(cfg.batch):
+        _assert_same_sets(got[b], oracle.topk(sc[b], cfg.topk))
+        rows = [r for r in band_rows if rb <= r < re_]
+        ref = _oracle_scores(cfg, inp, b, rows)
+        check_topk_band(got[b][np.asarray(rows) - rb], ref, cfg.topk)
 
 
 def test_indexer_topk_equals_two_pass_4k():
@@ -186,7 +200,9 @@ def test_indexer_topk_ragged(n, kvl, pos0, rb, re_):
     inp["kv_len"][:] = torch.tensor([kvl, max(1, kvl - 9)], dtype=torch.int32)
     inp["q_pos0"][:] = torch.tensor([pos0, pos0 + 1], dtype=torch.int32)
     g = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
-    _assert_same_sets(_fused(cfg, g, rb, re_), _two_pass(cfg, g, rb, re_))
+    fused = _fused(cfg, g, rb, re_)
+    _assert_same_sets(fused, _two_pass(cfg, g, rb, re_))
+    _check_fused_against_oracle(cfg, inp, g, rb, re_, fused, [rb, rb + 1, (rb + re_) // 2, re_ - 1])
 
 
 def test_indexer_topk_all_ties_take_lowest_indices():
@@ -199,6 +215,7 @@ def test_indexer_topk_all_ties_take_lowest_indices():
     _assert_same_sets(fused, _two_pass(cfg, g, 2400, 3000))
     got = np.sort(fused.cpu().numpy()[0][100:], axis=-1)
     assert np.array_equal(got, np.broadcast_to(np.arange(2048, dtype=np.int32), got.shape))
+    _check_fused_against_oracle(cfg, inp, g, 2400, 3000, fused, [2400, 2499, 2500, 2999])
 
 
 def test_indexer_topk_rising_scores_force_compactions():
@@ -215,7 +232,9 @@ def test_indexer_topk_rising_scores_force_compactions():
     inp["k_scale"] = inp["k_scale"] * (1.0 + torch.arange(cfg.n_kv, dtype=torch.float32) / 64.0)
     g = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
     rb, re_ = cfg.n_q - 256, cfg.n_q
-    _assert_same_sets(_fused(cfg, g, rb, re_), _two_pass(cfg, g, rb, re_))
+    fused = _fused(cfg, g, rb, re_)
+    _assert_same_sets(fused, _two_pass(cfg, g, rb, re_))
+    _check_fused_against_oracle(cfg, inp, g, rb, re_, fused, [rb, rb + 127, re_ - 1])
 
 
 # ------------------------------------------------------------------ attention
@@ -285,6 +304,31 @@ def test_forward_decode_32k_sampled_sequences():
     res = dsa.forward(g, cfg)
     dsa.dsa_check()
     for b in (0, 21, 63):
+        ref_s = _oracle_scores(cfg, inp, b, [0])
+        gidx = res["indices"][b].cpu().numpy()
+        check_topk_band(gidx, ref_s, cfg.topk)
+        o_ref, l_ref = _oracle_attn(cfg, inp, b, [0], gidx)
+        check_attn(res["out"][b].cpu().numpy(), o_ref, res["lse"][b].cpu().numpy(), l_ref)
+
+
+# rows of the k boundary, 128-row tile edges, mid-sequence and the last row
+SAMPLE_16K = [0, 1, 127, 128, 2046, 2047, 2048, 2049, 4095, 4096, 8191, 8192, 12345, 16256,
+              16383]
+
+
+def test_forward_16k_sampled_rows():
+    """Prefill at L = 16384 through dsa_forward (the fused indexer + top-k,
+    then the attention), the launches the bench times."""
+    cfg, inp, g = _inputs("prefill_16k", device="cuda")
+    _check_forward(cfg, inp, g, 0, np.array(SAMPLE_16K))
+
+
+def test_forward_decode_64k_sampled_sequences():
+    """Batch decode, 64 sequences x 65536 cached tokens, through dsa_forward."""
+    cfg, inp, g = _inputs("decode_64k", device="cuda")
+    res = dsa.forward(g, cfg)
+    dsa.dsa_check()
+    for b in (0, 1, 31, 62, 63):
         ref_s = _oracle_scores(cfg, inp, b, [0])
         gidx = res["indices"][b].cpu().numpy()
         check_topk_band(gidx, ref_s, cfg.topk)
