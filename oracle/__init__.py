@@ -49,6 +49,8 @@ def _load():
         lib.oracle_topk.argtypes = [I, I, I, P, P, I]
         lib.oracle_sparse_attn.argtypes = [I, I, I, I, I, I, ctypes.c_double,
                                            P, P, P, P, P, I]
+        lib.oracle_indexer_kl.argtypes = [I, I, I, I, P, P, P, P, P, P, I, I, I,
+                                          ctypes.c_double, P, P, P, P, P, P, I]
         _lib = lib
     return _lib
 
@@ -140,6 +142,32 @@ def sparse_attn(q, kv, idx, scale, v_dim, n_threads=0):
     _load().oracle_sparse_attn(n, S, H, Dqk, int(v_dim), k, float(scale), _ptr(q),
                                _ptr(kv), _ptr(idx), _ptr(o), _ptr(lse), int(n_threads))
     return o, lse
+
+
+def indexer_kl(q8, qs, w, k8, ks, pos, kv_len, q, kv, scale, n_threads=0):
+    """Indexer warm-up loss and gradient (see oracle.cpp, oracle_indexer_kl)
+    for rows q8 [n, HI, DI], qs/w [n, HI], pos [n], main queries q [n, H, Dqk]
+    (bf16) against keys k8 [S, DI], ks [S] and latent rows kv [S, Dqk].
+
+    Returns dict(loss [n], dw [n, HI], dq [n, HI, DI], dk [S, DI]), float64;
+    dq / dk are gradients with respect to the dequantised indexer vectors.
+    """
+    q8 = _np(q8, np.uint8); k8 = _np(k8, np.uint8)
+    qs = _np(qs, np.float32); w = _np(w, np.float32); ks = _np(ks, np.float32)
+    pos = _np(pos, np.int32); q = _np(q, np.uint16); kv = _np(kv, np.uint16)
+    n, HI, DI = q8.shape
+    S = k8.shape[0]
+    _, H, Dqk = q.shape
+    assert k8.shape == (S, DI) and qs.shape == (n, HI) and w.shape == (n, HI)
+    assert ks.shape == (S,) and pos.shape == (n,) and q.shape[0] == n and kv.shape == (S, Dqk)
+    loss = np.empty(n, dtype=np.float64)
+    dw = np.empty((n, HI), dtype=np.float64)
+    dq = np.empty((n, HI, DI), dtype=np.float64)
+    dk = np.empty((S, DI), dtype=np.float64)
+    _load().oracle_indexer_kl(n, S, HI, DI, _ptr(q8), _ptr(qs), _ptr(w), _ptr(k8), _ptr(ks),
+                              _ptr(pos), int(kv_len), H, Dqk, float(scale), _ptr(q), _ptr(kv),
+                              _ptr(loss), _ptr(dw), _ptr(dq), _ptr(dk), int(n_threads))
+    return {"loss": loss, "dw": dw, "dq": dq, "dk": dk}
 
 
 def forward(inp, cfg, b=0, rows=None, n_threads=0):

@@ -13,6 +13,8 @@
 //     the lower key index, fewer than k valid keys -> all of them, pad -1;
 //   * the per-row FP8 encoding of the indexer inputs (scale = amax / 448,
 //     nearest E4M3 value, ties to even, saturating);
+//   * the indexer's dense warm-up loss KL(p || Softmax(I)) and its gradient
+//     (section "预训练策略 / 密集预热阶段"), see oracle_indexer_kl;
 //   * the attention over the selected latent rows c_s (MQA: every query head
 //     reads the same row; K = all qk_dim dims, V = the first v_dim dims; the
 //     latent width 576 = 512 + 64 follows the MLA section 1.1 of page
@@ -244,6 +246,121 @@ void oracle_sparse_attn(int n_rows, int S, int H, int Dqk, int Dv, int k,
       lse[static_cast<size_t>(r) * H + h] = m + std::log(l);
     }
   });
+}
+
+// Indexer warm-up loss and its gradient for n_rows query rows of ONE
+// sequence (page "DeepseekV3.2 拆解", section "预训练策略 / 密集预热阶段":
+// the main model is frozen and the indexer alone is trained to match the
+// dense attention distribution, L^I = sum_t KL(p_{t,:} || Softmax(I_{t,:}))).
+//
+// Readings taken where the page is silent:
+//   * p_{t,:} is the main attention's dense causal softmax over the visible
+//     keys (s <= pos[t], s < kv_len), averaged over the H query heads (each
+//     head's softmax sums to one, so the mean is one distribution per query);
+//   * Softmax(I_{t,:}) runs over the same visible keys;
+//   * gradients are taken with respect to w and to the dequantised indexer
+//     vectors q^ = code * q_scale and k^ = code * k_scale (the FP8 encoding is
+//     upstream of the indexer and passes the gradient through unchanged).
+// With r_t = Softmax(I_{t,:}) and g[t,s] = r_t[s] - p[t,s] (the derivative of
+// KL(p || Softmax(I)) with respect to I[t,s] when p sums to one), and
+// x[t,j,s] = q^[t,j] . k^[s]:
+//   dL/dw[t,j]  = sum_s g[t,s] ReLU(x[t,j,s])
+//   dL/dq^[t,j] = sum_s g[t,s] w[t,j] [x[t,j,s] > 0] k^[s]
+//   dL/dk^[s]   = sum_t sum_j g[t,s] w[t,j] [x[t,j,s] > 0] q^[t,j]
+//   q8, qs, w, k8, ks, pos, kv_len  as oracle_indexer_scores
+//   q   [n_rows, H, Dqk] bf16 bits (main attention queries), kv [S, Dqk] bf16
+//   loss [n_rows] (KL of each row), dw [n_rows, HI], dq [n_rows, HI, DI],
+//   dk [S, DI] (summed over the given rows; zero where no row sees the key)
+void oracle_indexer_kl(int n_rows, int S, int HI, int DI, const uint8_t* q8, const float* qs,
+                       const float* w, const uint8_t* k8, const float* ks, const int32_t* pos,
+                       int kv_len, int H, int Dqk, double scale, const uint16_t* q,
+                       const uint16_t* kv, double* loss, double* dw, double* dq, double* dk,
+                       int n_threads) {
+  std::vector<double> khat(static_cast<size_t>(S) * DI);
+  for (int s = 0; s < S; ++s)
+    for (int d = 0; d < DI; ++d)
+      khat[static_cast<size_t>(s) * DI + d] =
+          e4m3_value(k8[static_cast<size_t>(s) * DI + d]) * static_cast<double>(ks[s]);
+  // per-row contributions to dk, summed after the parallel part
+  std::vector<double> dk_rows(static_cast<size_t>(n_rows) * S * DI, 0.0);
+  parallel_rows(n_rows, n_threads, [&](int r) {
+    const int n_vis = std::max(0, std::min(pos[r] + 1, std::min(kv_len, S)));
+    std::vector<double> qhat(static_cast<size_t>(HI) * DI);
+    for (int j = 0; j < HI; ++j)
+      for (int d = 0; d < DI; ++d)
+        qhat[static_cast<size_t>(j) * DI + d] =
+            e4m3_value(q8[(static_cast<size_t>(r) * HI + j) * DI + d]) *
+            static_cast<double>(qs[static_cast<size_t>(r) * HI + j]);
+    double* dw_r = dw + static_cast<size_t>(r) * HI;
+    double* dq_r = dq + static_cast<size_t>(r) * HI * DI;
+    for (int i = 0; i < HI; ++i) dw_r[i] = 0.0;
+    for (int i = 0; i < HI * DI; ++i) dq_r[i] = 0.0;
+    loss[r] = 0.0;
+    if (n_vis == 0) return;
+    // p: dense causal attention of each head over the visible keys, averaged
+    std::vector<double> p(n_vis, 0.0), z(n_vis), qh(Dqk);
+    for (int h = 0; h < H; ++h) {
+      for (int d = 0; d < Dqk; ++d)
+        qh[d] = bf16_value(q[(static_cast<size_t>(r) * H + h) * Dqk + d]);
+      double m = -std::numeric_limits<double>::infinity();
+      for (int s = 0; s < n_vis; ++s) {
+        double dot = 0.0;
+        for (int d = 0; d < Dqk; ++d)
+          dot += qh[d] * bf16_value(kv[static_cast<size_t>(s) * Dqk + d]);
+        z[s] = scale * dot;
+        m = std::max(m, z[s]);
+      }
+      double l = 0.0;
+      for (int s = 0; s < n_vis; ++s) {
+        z[s] = std::exp(z[s] - m);
+        l += z[s];
+      }
+      for (int s = 0; s < n_vis; ++s) p[s] += z[s] / l / static_cast<double>(H);
+    }
+    // indexer scores I (direct form) and x kept for the gradient
+    std::vector<double> x(static_cast<size_t>(n_vis) * HI), I(n_vis);
+    for (int s = 0; s < n_vis; ++s) {
+      double score = 0.0;
+      for (int j = 0; j < HI; ++j) {
+        double dot = 0.0;
+        for (int d = 0; d < DI; ++d)
+          dot += qhat[static_cast<size_t>(j) * DI + d] * khat[static_cast<size_t>(s) * DI + d];
+        x[static_cast<size_t>(s) * HI + j] = dot;
+        score += static_cast<double>(w[static_cast<size_t>(r) * HI + j]) * (dot > 0.0 ? dot : 0.0);
+      }
+      I[s] = score;
+    }
+    // log Softmax(I) and the KL divergence
+    double mi = -std::numeric_limits<double>::infinity();
+    for (int s = 0; s < n_vis; ++s) mi = std::max(mi, I[s]);
+    double li = 0.0;
+    for (int s = 0; s < n_vis; ++s) li += std::exp(I[s] - mi);
+    const double lse_i = mi + std::log(li);
+    double kl = 0.0;
+    for (int s = 0; s < n_vis; ++s)
+      if (p[s] > 0.0) kl += p[s] * (std::log(p[s]) - (I[s] - lse_i));
+    loss[r] = kl;
+    // gradient
+    double* dk_r = dk_rows.data() + static_cast<size_t>(r) * S * DI;
+    for (int s = 0; s < n_vis; ++s) {
+      const double g = std::exp(I[s] - lse_i) - p[s];
+      for (int j = 0; j < HI; ++j) {
+        const double xv = x[static_cast<size_t>(s) * HI + j];
+        if (xv <= 0.0) continue;
+        const double wj = static_cast<double>(w[static_cast<size_t>(r) * HI + j]);
+        dw_r[j] += g * xv;
+        for (int d = 0; d < DI; ++d) {
+          dq_r[static_cast<size_t>(j) * DI + d] += g * wj * khat[static_cast<size_t>(s) * DI + d];
+          dk_r[static_cast<size_t>(s) * DI + d] += g * wj * qhat[static_cast<size_t>(j) * DI + d];
+        }
+      }
+    }
+  });
+  for (size_t i = 0; i < static_cast<size_t>(S) * DI; ++i) {
+    double acc = 0.0;
+    for (int r = 0; r < n_rows; ++r) acc += dk_rows[static_cast<size_t>(r) * S * DI + i];
+    dk[i] = acc;
+  }
 }
 
 }  // extern "C"

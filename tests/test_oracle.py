@@ -365,3 +365,156 @@ def test_forward_tiny_invariants(oracle_lib):
         p = torch.softmax(qd @ kd.T * cfg.softmax_scale, -1)
         np.testing.assert_allclose(res["o"][r], (p @ kd[:, : cfg.v_dim]).numpy(), rtol=0, atol=1e-12)
     assert len(dense_rows) > 0
+
+
+# ---------------------------------------------------------------- warm-up loss
+# Page "DeepseekV3.2 拆解", section "预训练策略 / 密集预热阶段": the indexer
+# is trained against the dense attention distribution with
+# L^I = sum_t KL(p_{t,:} || Softmax(I_{t,:})).
+
+def _bf16_bits(vals):
+    return torch.tensor(vals, dtype=torch.float32).to(torch.bfloat16)
+
+
+def test_kl_two_key_case_by_hand(oracle_lib):
+    """Two query rows over two keys, one main head, one indexer head of one
+    dim, every value exact in bf16 / e4m3. Row 0 sees only key 0: both
+    distributions are [1], so its loss and gradient vanish. Row 1: the main
+    logits are (0, a) and the indexer scores (0, b) with b = w q^ k^_1, so
+    p = (1, e^a) / (1 + e^a), r = (1, e^b) / (1 + e^b); x_0 = 0 contributes
+    neither to I nor to the gradient (ReLU and its mask are both zero)."""
+    scale, wv, qsv, ks1 = 0.75, 1.5, 2.0, 0.5
+    q = _bf16_bits([[[1.0, 0.0]], [[1.0, 0.0]]])              # [2 rows, 1 head, 2]
+    kv = _bf16_bits([[0.0, 0.0], [1.0, 0.0]])                 # c_0 = 0, c_1 = e_0
+    one = 0x38                                                # e4m3 code of 1.0
+    q8 = torch.tensor([[[one]], [[one]]], dtype=torch.uint8)  # [2, 1, 1]
+    k8 = torch.tensor([[0x00], [one]], dtype=torch.uint8)     # k^_0 = 0, k^_1 = ks1
+    qs = torch.full((2, 1), qsv)
+    w = torch.full((2, 1), wv)
+    ks = torch.tensor([1.0, ks1])
+    res = oracle_lib.indexer_kl(q8, qs, w, k8, ks, np.array([0, 1], np.int32), 2, q, kv, scale)
+    a = scale * 1.0
+    xq = qsv * ks1                                            # x[1, 0, 1] = q^ . k^_1
+    b = wv * xq
+    p1 = math.exp(a) / (1 + math.exp(a))
+    r1 = math.exp(b) / (1 + math.exp(b))
+    p0, r0 = 1 - p1, 1 - r1
+    want = p0 * math.log(p0 / r0) + p1 * math.log(p1 / r1)
+    g1 = r1 - p1
+    assert res["loss"][0] == 0.0 and (res["dw"][0] == 0).all() and (res["dq"][0] == 0).all()
+    assert abs(res["loss"][1] - want) < 1e-14
+    assert abs(res["dw"][1, 0] - g1 * xq) < 1e-14
+    assert abs(res["dq"][1, 0, 0] - g1 * wv * ks1) < 1e-14
+    assert abs(res["dk"][1, 0] - g1 * wv * qsv) < 1e-14
+    assert res["dk"][0, 0] == 0.0
+
+
+def _kl_case(seed, n=20, HI=4, DI=32, H=8, Dqk=64, kv_len=None, w_scale=0.5):
+    q8, qs, w, k8, ks = _small_indexer(seed, n, n, HI, DI)
+    g = torch.Generator().manual_seed(seed + 1)
+    q = (torch.randn(n, H, Dqk, generator=g) * 0.5).to(torch.bfloat16)
+    kv = torch.randn(n, Dqk, generator=g).to(torch.bfloat16)
+    return dict(q8=q8, qs=qs, w=w * w_scale, k8=k8, ks=ks, pos=np.arange(n, dtype=np.int32),
+                kv_len=n if kv_len is None else kv_len, q=q, kv=kv, scale=0.125)
+
+
+def _kl(oracle_lib, c, **over):
+    d = dict(c, **over)
+    return oracle_lib.indexer_kl(d["q8"], d["qs"], d["w"], d["k8"], d["ks"], d["pos"],
+                                 d["kv_len"], d["q"], d["kv"], d["scale"])
+
+
+def test_kl_matches_library_kl_div_and_is_nonnegative(oracle_lib):
+    """Given the (separately pinned) indexer scores, the loss is torch's
+    kl_div of log_softmax(I) against the head-averaged causal softmax of the
+    main logits (torch softmax over masked float64 logits)."""
+    c = _kl_case(3)
+    res = _kl(oracle_lib, c)
+    n = len(c["pos"])
+    sc = oracle_lib.indexer_scores(c["q8"], c["qs"], c["w"], c["k8"], c["ks"], c["pos"], n)
+    I = torch.from_numpy(sc)
+    qd, kd = c["q"].double(), c["kv"].double()
+    z = torch.einsum("thd,sd->ths", qd, kd) * c["scale"]
+    mask = torch.triu(torch.ones(n, n, dtype=torch.bool), 1)
+    p = torch.softmax(z.masked_fill(mask[:, None, :], -math.inf), -1).mean(1)
+    for t in range(n):
+        want = torch.nn.functional.kl_div(torch.log_softmax(I[t, : t + 1], -1), p[t, : t + 1],
+                                          reduction="sum").item()
+        assert abs(res["loss"][t] - want) < 1e-12
+    assert (res["loss"] >= -1e-15).all() and res["loss"][1:].max() > 1e-3
+
+
+def test_kl_vanishes_when_both_distributions_are_uniform(oracle_lib):
+    """w = 0 makes every indexer score 0 and q = 0 every main logit 0: both
+    distributions are uniform over the visible keys, loss and gradient 0."""
+    c = _kl_case(4)
+    res = _kl(oracle_lib, c, w=torch.zeros_like(c["w"]), q=torch.zeros_like(c["q"]))
+    # zero up to the rounding of 1/n against the mean of H equal 1/n values
+    assert np.abs(res["loss"]).max() < 1e-14
+    assert np.abs(res["dw"]).max() < 1e-12 and np.abs(res["dq"]).max() < 1e-12
+    assert np.abs(res["dk"]).max() < 1e-12
+
+
+def test_kl_gradient_of_w_by_central_differences(oracle_lib):
+    c = _kl_case(5)
+    res = _kl(oracle_lib, c)
+    eps = 1e-6
+    for (t, j) in [(1, 0), (7, 3), (19, 2), (12, 1)]:
+        wp, wm = c["w"].clone(), c["w"].clone()
+        wp[t, j] += eps
+        wm[t, j] -= eps
+        # the fp32 w cannot hold w +- 1e-6 exactly: difference by the actual step
+        h = float(wp[t, j]) - float(wm[t, j])
+        fd = (_kl(oracle_lib, c, w=wp)["loss"].sum() - _kl(oracle_lib, c, w=wm)["loss"].sum()) / h
+        assert abs(fd - res["dw"][t, j]) <= 1e-6 * max(1.0, abs(res["dw"][t, j])), (t, j)
+
+
+def test_kl_gradient_along_the_scales_by_central_differences(oracle_lib):
+    """q^[t,j] = code * q_scale[t,j]: d loss / d q_scale[t,j] = dq[t,j] . code;
+    likewise for k_scale[s] and dk[s]."""
+    c = _kl_case(6)
+    res = _kl(oracle_lib, c)
+    dec_q = _decode_fp8_torch(c["q8"]).numpy()
+    dec_k = _decode_fp8_torch(c["k8"]).numpy()
+    rel = 2e-6
+    for (t, j) in [(3, 1), (15, 0), (19, 3)]:
+        qp, qm = c["qs"].clone(), c["qs"].clone()
+        qp[t, j] *= 1 + rel
+        qm[t, j] *= 1 - rel
+        h = float(qp[t, j]) - float(qm[t, j])
+        fd = (_kl(oracle_lib, c, qs=qp)["loss"].sum() - _kl(oracle_lib, c, qs=qm)["loss"].sum()) / h
+        want = float(res["dq"][t, j] @ dec_q[t, j])
+        assert abs(fd - want) <= 1e-5 * max(1.0, abs(want)), (t, j)
+    for s in [0, 4, 11, 19]:
+        kp, km = c["ks"].clone(), c["ks"].clone()
+        kp[s] *= 1 + rel
+        km[s] *= 1 - rel
+        h = float(kp[s]) - float(km[s])
+        fd = (_kl(oracle_lib, c, ks=kp)["loss"].sum() - _kl(oracle_lib, c, ks=km)["loss"].sum()) / h
+        want = float(res["dk"][s] @ dec_k[s])
+        assert abs(fd - want) <= 1e-5 * max(1.0, abs(want)), s
+
+
+def test_kl_gradients_match_autograd(oracle_lib):
+    """Element-wise dq^ and dk^ (and dw) against torch autograd of the loss
+    written with library ops on the dequantised vectors, with a kv_len cut."""
+    n, HI = 20, 4
+    c = _kl_case(7, n=n, HI=HI, kv_len=16)
+    res = _kl(oracle_lib, c)
+    qh = (_decode_fp8_torch(c["q8"]) * c["qs"].double()[..., None]).requires_grad_()
+    kh = (_decode_fp8_torch(c["k8"]) * c["ks"].double()[:, None]).requires_grad_()
+    w = c["w"].double().requires_grad_()
+    x = torch.einsum("tjd,sd->tjs", qh, kh)
+    I = torch.einsum("tj,tjs->ts", w, torch.relu(x))
+    z = torch.einsum("thd,sd->ths", c["q"].double(), c["kv"].double()) * c["scale"]
+    s_idx = torch.arange(n)
+    vis = (s_idx[None, :] <= s_idx[:, None]) & (s_idx[None, :] < c["kv_len"])
+    p = torch.softmax(z.masked_fill(~vis[:, None, :], -math.inf), -1).mean(1)
+    logr = torch.log_softmax(I.masked_fill(~vis, -math.inf), -1)
+    terms = torch.where(vis & (p > 0), p * (torch.log(p) - logr), torch.zeros_like(p))
+    terms.sum().backward()
+    np.testing.assert_allclose(res["loss"], terms.sum(-1).detach().numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(res["dw"], w.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(res["dq"], qh.grad.numpy(), rtol=0, atol=1e-11)
+    np.testing.assert_allclose(res["dk"], kh.grad.numpy(), rtol=0, atol=1e-11)
+    assert (res["dk"][16:] == 0).all()      # keys past kv_len see no row
