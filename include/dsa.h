@@ -88,6 +88,38 @@ typedef struct {
 } dsa_shape;
 
 /*
+ * Where the keys and the query positions of a call live. Every call below
+ * has an _ex variant that takes a `const dsa_layout*` right after the shape;
+ * NULL (and the plain call) means contiguous caches and consecutive rows.
+ *
+ * Paged caches (the PagedAttention layout, page "DeepSeek-V3 MoE blog",
+ * section 4.1): with block_table set, the key inputs k_fp8, k_scale and kv
+ * are POOLS of pool_rows rows, and logical key s of sequence b is pool row
+ *     block_table[b * max_pages + s / page_size] * page_size + s % page_size.
+ * Indices (dsa_topk's output, dsa_sparse_attn's input) stay logical key
+ * positions. Every page that kv_len[b] (or n_kv) reaches must be mapped. A
+ * page outside [0, pool_rows / page_size) is not read: its keys count as
+ * zero vectors, and the next dsa_check() returns DSA_ERR_INVALID_ARG.
+ *
+ * Explicit query positions: with row_pos set, query row i of sequence b sits
+ * at absolute position row_pos[b * n_q + i] (visibility: s <= row_pos and
+ * s < kv_len), instead of q_pos0[b] + i. This lets the query rows of one
+ * prefill be split over several calls or GPUs in any grouping; the fused
+ * indexer treats every 4 consecutive rows of the call as one tile group, so
+ * keep rows of nearby positions together and in increasing order for speed
+ * (any order is correct).
+ */
+typedef struct {
+  const int32_t* row_pos;      /* [B, n_q] device int32, or NULL               */
+  const int32_t* block_table;  /* [B, max_pages] device int32, or NULL         */
+  int32_t max_pages;           /* row stride of block_table,
+                                  >= ceil(n_kv / page_size)                    */
+  int32_t page_size;           /* keys per page: power of two in [128, 65536]  */
+  int64_t pool_rows;           /* rows of the key pools: a multiple of
+                                  page_size, below 2^31 - 256                  */
+} dsa_layout;
+
+/*
  * Indexer scores (page "DeepseekV3.2 拆解", eq. I_{t,s}), materialised.
  *   q_fp8   [B, n_q, H^I, d^I] e4m3fn codes     q_scale [B, n_q, H^I] fp32
  *   w       [B, n_q, H^I] fp32 head weights
@@ -106,6 +138,12 @@ dsa_status dsa_indexer_scores(const dsa_shape* shape, const uint8_t* q_fp8,
                               const int32_t* q_pos0, const int32_t* kv_len,
                               int32_t row_begin, int32_t row_end,
                               int32_t flags, float* scores, void* stream);
+dsa_status dsa_indexer_scores_ex(const dsa_shape* shape, const dsa_layout* layout,
+                                 const uint8_t* q_fp8, const float* q_scale, const float* w,
+                                 const uint8_t* k_fp8, const float* k_scale,
+                                 const int32_t* q_pos0, const int32_t* kv_len,
+                                 int32_t row_begin, int32_t row_end, int32_t flags,
+                                 float* scores, void* stream);
 
 /*
  * Per-row FP8 quantisation of the indexer inputs (page "DeepseekV3.2 拆解",
@@ -146,6 +184,12 @@ dsa_status dsa_indexer_topk(const dsa_shape* shape, const uint8_t* q_fp8,
                             const int32_t* q_pos0, const int32_t* kv_len,
                             int32_t row_begin, int32_t row_end, int32_t* indices,
                             void* stream);
+dsa_status dsa_indexer_topk_ex(const dsa_shape* shape, const dsa_layout* layout,
+                               const uint8_t* q_fp8, const float* q_scale, const float* w,
+                               const uint8_t* k_fp8, const float* k_scale,
+                               const int32_t* q_pos0, const int32_t* kv_len,
+                               int32_t row_begin, int32_t row_end, int32_t* indices,
+                               void* stream);
 
 /*
  * Top-k selection per score row (page "DeepseekV3.2 拆解", eq. u_t: keep the
@@ -163,6 +207,11 @@ dsa_status dsa_topk(const dsa_shape* shape, const float* scores,
                     int32_t row_begin, int32_t row_end,
                     const int32_t* q_pos0, const int32_t* kv_len,
                     int32_t* indices, void* ws, size_t ws_bytes, void* stream);
+/* Only layout->row_pos matters here (scores are logical key positions). */
+dsa_status dsa_topk_ex(const dsa_shape* shape, const dsa_layout* layout, const float* scores,
+                       int32_t row_begin, int32_t row_end,
+                       const int32_t* q_pos0, const int32_t* kv_len,
+                       int32_t* indices, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Sparse MQA attention over the selected latent rows (eq. u_t).
@@ -183,6 +232,11 @@ dsa_status dsa_sparse_attn(const dsa_shape* shape, const uint16_t* q,
                            const uint16_t* kv, const int32_t* indices,
                            void* out, int32_t out_dtype, float* lse,
                            void* ws, size_t ws_bytes, void* stream);
+/* Only layout->block_table (and its sizes) matters here. */
+dsa_status dsa_sparse_attn_ex(const dsa_shape* shape, const dsa_layout* layout,
+                              const uint16_t* q, const uint16_t* kv, const int32_t* indices,
+                              void* out, int32_t out_dtype, float* lse,
+                              void* ws, size_t ws_bytes, void* stream);
 
 /*
  * dsa_sparse_attn without a caller-provided workspace. The paper has no
@@ -233,6 +287,13 @@ dsa_status dsa_forward(const dsa_shape* shape, const uint8_t* q_fp8,
                        const uint16_t* q, const uint16_t* kv,
                        int32_t* indices_out, void* out, int32_t out_dtype,
                        float* lse, void* ws, size_t ws_bytes, void* stream);
+dsa_status dsa_forward_ex(const dsa_shape* shape, const dsa_layout* layout,
+                          const uint8_t* q_fp8, const float* q_scale, const float* w,
+                          const uint8_t* k_fp8, const float* k_scale,
+                          const int32_t* q_pos0, const int32_t* kv_len,
+                          const uint16_t* q, const uint16_t* kv,
+                          int32_t* indices_out, void* out, int32_t out_dtype,
+                          float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* Rows per indexer/top-k step that dsa_forward uses for this shape. With
  * the fused plan it is n_q (one dsa_indexer_topk launch over all rows, no
@@ -260,7 +321,8 @@ dsa_status dsa_workspace_size(const dsa_shape* shape, int32_t op,
                               size_t* bytes);
 
 /* Synchronises `stream`, then returns DSA_ERR_CUDA for a pending CUDA error,
- * DSA_ERR_TIMEOUT if a kernel's bounded wait ran out since the last check
+ * DSA_ERR_TIMEOUT if a kernel's bounded wait ran out since the last check,
+ * DSA_ERR_INVALID_ARG if a kernel met a block-table page outside its pool
  * (the error word is cleared), else DSA_OK. */
 dsa_status dsa_check(void* stream);
 

@@ -50,6 +50,27 @@ class DsaShape(ctypes.Structure):
                 ("softmax_scale", ctypes.c_float)]
 
 
+class DsaLayout(ctypes.Structure):
+    """dsa_layout: explicit query positions and / or a paged key cache."""
+    _fields_ = [("row_pos", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
+                ("max_pages", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("pool_rows", ctypes.c_int64)]
+
+
+def make_layout(row_pos=None, block_table=None, page_size=0, pool_rows=0):
+    """A DsaLayout from CUDA tensors: row_pos [B, n_q] int32 and/or
+    block_table [B, max_pages] int32 with the pool geometry. The tensors must
+    outlive every call that uses the layout."""
+    lay = DsaLayout()
+    lay.row_pos = _ptr(row_pos, _dt()["i32"], "row_pos")
+    if block_table is not None:
+        lay.block_table = _ptr(block_table, _dt()["i32"], "block_table")
+        lay.max_pages = int(block_table.shape[-1])
+        lay.page_size = int(page_size)
+        lay.pool_rows = int(pool_rows)
+    return lay
+
+
 _lib = None
 
 
@@ -84,13 +105,20 @@ def load_library(path: str | None = None):
     lib.dsa_forward_chunk_rows.argtypes = [SP, ctypes.POINTER(I32)]
     lib.dsa_forward_plan.argtypes = [SP, ctypes.POINTER(I32), ctypes.POINTER(I32),
                                      ctypes.POINTER(I32)]
+    LP = ctypes.POINTER(DsaLayout)
+    lib.dsa_indexer_scores_ex.argtypes = [SP, LP, P, P, P, P, P, P, P, I32, I32, I32, P, P]
+    lib.dsa_indexer_topk_ex.argtypes = [SP, LP, P, P, P, P, P, P, P, I32, I32, P, P]
+    lib.dsa_topk_ex.argtypes = [SP, LP, P, I32, I32, P, P, P, P, SZ, P]
+    lib.dsa_sparse_attn_ex.argtypes = [SP, LP, P, P, P, P, I32, P, P, SZ, P]
+    lib.dsa_forward_ex.argtypes = [SP, LP, P, P, P, P, P, P, P, P, P, P, P, I32, P, P, SZ, P]
     lib.dsa_status_string.argtypes = [ctypes.c_int]
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_last_error.restype = ctypes.c_char_p
     lib.dsa_version.restype = ctypes.c_char_p
     for fn in ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
                "dsa_workspace_size", "dsa_check", "dsa_forward_chunk_rows",
-               "dsa_sparse_attn_noalloc", "dsa_forward_plan"):
+               "dsa_sparse_attn_noalloc", "dsa_forward_plan", "dsa_indexer_scores_ex",
+               "dsa_indexer_topk_ex", "dsa_topk_ex", "dsa_sparse_attn_ex", "dsa_forward_ex"):
         getattr(lib, fn).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -122,6 +150,10 @@ def _ptr(t, dtype=None, what="tensor"):
     if dtype is not None and t.dtype not in dtype:
         raise ValueError(f"{what} has dtype {t.dtype}, expected one of {dtype}")
     return t.data_ptr()
+
+
+def _lay(layout):
+    return ctypes.byref(layout) if layout is not None else None
 
 
 def _stream(stream):
@@ -160,10 +192,11 @@ def forward_plan(shape: DsaShape) -> dict:
 
 
 def dsa_indexer_scores(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
-                       row_begin, row_end, scores, stream=None, flags=DSA_SCORES_ALL):
+                       row_begin, row_end, scores, stream=None, flags=DSA_SCORES_ALL,
+                       layout=None):
     d = _dt()
-    _raise(load_library().dsa_indexer_scores(
-        ctypes.byref(shape), _ptr(q_fp8, d["u8"], "q_fp8"), _ptr(q_scale, d["f32"], "q_scale"),
+    _raise(load_library().dsa_indexer_scores_ex(
+        ctypes.byref(shape), _lay(layout), _ptr(q_fp8, d["u8"], "q_fp8"), _ptr(q_scale, d["f32"], "q_scale"),
         _ptr(w, d["f32"], "w"), _ptr(k_fp8, d["u8"], "k_fp8"), _ptr(k_scale, d["f32"], "k_scale"),
         _ptr(q_pos0, d["i32"], "q_pos0"), _ptr(kv_len, d["i32"], "kv_len"),
         int(row_begin), int(row_end), int(flags), _ptr(scores, d["f32"], "scores"),
@@ -171,10 +204,10 @@ def dsa_indexer_scores(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
 
 
 def dsa_indexer_topk(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
-                     row_begin, row_end, indices, stream=None):
+                     row_begin, row_end, indices, stream=None, layout=None):
     d = _dt()
-    _raise(load_library().dsa_indexer_topk(
-        ctypes.byref(shape), _ptr(q_fp8, d["u8"], "q_fp8"), _ptr(q_scale, d["f32"], "q_scale"),
+    _raise(load_library().dsa_indexer_topk_ex(
+        ctypes.byref(shape), _lay(layout), _ptr(q_fp8, d["u8"], "q_fp8"), _ptr(q_scale, d["f32"], "q_scale"),
         _ptr(w, d["f32"], "w"), _ptr(k_fp8, d["u8"], "k_fp8"), _ptr(k_scale, d["f32"], "k_scale"),
         _ptr(q_pos0, d["i32"], "q_pos0"), _ptr(kv_len, d["i32"], "kv_len"),
         int(row_begin), int(row_end), _ptr(indices, d["i32"], "indices"), _stream(stream)))
@@ -204,21 +237,22 @@ def dsa_selftest_wait_timeout(limit_ms=100, stream=None):
 
 
 def dsa_topk(shape, scores, row_begin, row_end, q_pos0, kv_len, indices, ws=None,
-             ws_bytes=0, stream=None):
+             ws_bytes=0, stream=None, layout=None):
     d = _dt()
-    _raise(load_library().dsa_topk(
-        ctypes.byref(shape), _ptr(scores, d["f32"], "scores"), int(row_begin), int(row_end),
+    _raise(load_library().dsa_topk_ex(
+        ctypes.byref(shape), _lay(layout), _ptr(scores, d["f32"], "scores"), int(row_begin), int(row_end),
         _ptr(q_pos0, d["i32"], "q_pos0"), _ptr(kv_len, d["i32"], "kv_len"),
         _ptr(indices, d["i32"], "indices"), _ptr(ws, None, "ws"), int(ws_bytes),
         _stream(stream)))
 
 
-def dsa_sparse_attn(shape, q, kv, indices, out, lse=None, ws=None, ws_bytes=0, stream=None):
+def dsa_sparse_attn(shape, q, kv, indices, out, lse=None, ws=None, ws_bytes=0, stream=None,
+                    layout=None):
     import torch
     d = _dt()
     out_dtype = DSA_OUT_BF16 if out.dtype == torch.bfloat16 else DSA_OUT_F32
-    _raise(load_library().dsa_sparse_attn(
-        ctypes.byref(shape), _ptr(q, d["bf16"], "q"), _ptr(kv, d["bf16"], "kv"),
+    _raise(load_library().dsa_sparse_attn_ex(
+        ctypes.byref(shape), _lay(layout), _ptr(q, d["bf16"], "q"), _ptr(kv, d["bf16"], "kv"),
         _ptr(indices, d["i32"], "indices"), _ptr(out, (torch.float32, torch.bfloat16), "out"),
         out_dtype, _ptr(lse, d["f32"], "lse"), _ptr(ws, None, "ws"), int(ws_bytes),
         _stream(stream)))
@@ -237,12 +271,12 @@ def dsa_sparse_attn_noalloc(shape, q, kv, indices, out, lse=None, stream=None):
 
 
 def dsa_forward(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, q, kv,
-                indices_out, out, lse=None, ws=None, ws_bytes=0, stream=None):
+                indices_out, out, lse=None, ws=None, ws_bytes=0, stream=None, layout=None):
     import torch
     d = _dt()
     out_dtype = DSA_OUT_BF16 if out.dtype == torch.bfloat16 else DSA_OUT_F32
-    _raise(load_library().dsa_forward(
-        ctypes.byref(shape), _ptr(q_fp8, d["u8"], "q_fp8"), _ptr(q_scale, d["f32"], "q_scale"),
+    _raise(load_library().dsa_forward_ex(
+        ctypes.byref(shape), _lay(layout), _ptr(q_fp8, d["u8"], "q_fp8"), _ptr(q_scale, d["f32"], "q_scale"),
         _ptr(w, d["f32"], "w"), _ptr(k_fp8, d["u8"], "k_fp8"), _ptr(k_scale, d["f32"], "k_scale"),
         _ptr(q_pos0, d["i32"], "q_pos0"), _ptr(kv_len, d["i32"], "kv_len"),
         _ptr(q, d["bf16"], "q"), _ptr(kv, d["bf16"], "kv"),
@@ -264,7 +298,7 @@ def alloc_workspace(shape: DsaShape, op: int, device="cuda"):
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device), n
 
 
-def forward(inp: dict, cfg: DsaConfig, out_dtype=None, ws=None, stream=None):
+def forward(inp: dict, cfg: DsaConfig, out_dtype=None, ws=None, stream=None, layout=None):
     """Run the whole path on CUDA tensors from ``make_inputs``; returns
     dict(indices, out, lse). Output buffers are allocated with torch."""
     import torch
@@ -280,5 +314,6 @@ def forward(inp: dict, cfg: DsaConfig, out_dtype=None, ws=None, stream=None):
     else:
         n = ws.numel()
     dsa_forward(shape, inp["q_fp8"], inp["q_scale"], inp["w"], inp["k_fp8"], inp["k_scale"],
-                inp["q_pos0"], inp["kv_len"], inp["q"], inp["kv"], idx, out, lse, ws, n, stream)
+                inp["q_pos0"], inp["kv_len"], inp["q"], inp["kv"], idx, out, lse, ws, n, stream,
+                layout=layout)
     return {"indices": idx, "out": out, "lse": lse}

@@ -181,6 +181,45 @@ dsa_status check_attn_shape(const dsa_shape* s) {
   return DSA_OK;
 }
 
+// ------------------------------------------------------------------ layouts
+
+// Key rows and query positions of one call (dsa_layout, or the contiguous
+// default when it is NULL).
+struct HostLayout {
+  dsa::KeyMap km;
+  const int32_t* row_pos;
+};
+
+dsa_status resolve_layout(const dsa_shape* s, const dsa_layout* L, HostLayout* out) {
+  out->row_pos = L ? L->row_pos : nullptr;
+  out->km.block_table = nullptr;
+  out->km.max_pages = 0;
+  out->km.page_shift = 0;
+  out->km.pool_rows = static_cast<int64_t>(s->batch) * s->n_kv;
+  if (out->row_pos && reinterpret_cast<uintptr_t>(out->row_pos) % 4)
+    return fail(DSA_ERR_INVALID_ARG, "row_pos must be 4-byte aligned");
+  if (!L || !L->block_table) return DSA_OK;
+  const int32_t page = L->page_size;
+  if (page < 128 || page > 65536 || (page & (page - 1)))
+    return fail(DSA_ERR_INVALID_ARG, "page_size must be a power of two in [128, 65536] (got %d)",
+                page);
+  const int64_t need_pages = (static_cast<int64_t>(s->n_kv) + page - 1) / page;
+  if (L->max_pages < need_pages)
+    return fail(DSA_ERR_INVALID_ARG, "max_pages %d < ceil(n_kv / page_size) = %lld", L->max_pages,
+                static_cast<long long>(need_pages));
+  if (L->pool_rows < page || L->pool_rows % page != 0 || L->pool_rows > (1ll << 31) - 256)
+    return fail(DSA_ERR_INVALID_ARG,
+                "pool_rows must be a positive multiple of page_size below 2^31 - 256 (got %lld)",
+                static_cast<long long>(L->pool_rows));
+  if (reinterpret_cast<uintptr_t>(L->block_table) % 4)
+    return fail(DSA_ERR_INVALID_ARG, "block_table must be 4-byte aligned");
+  out->km.block_table = L->block_table;
+  out->km.max_pages = L->max_pages;
+  out->km.page_shift = __builtin_ctz(static_cast<unsigned>(page));
+  out->km.pool_rows = L->pool_rows;
+  return DSA_OK;
+}
+
 // ------------------------------------------------------------------ kernel attributes
 
 template <class K>
@@ -198,11 +237,11 @@ dsa_status set_smem(K kernel, int bytes, int dev, std::atomic<bool>* done_flags)
 // ------------------------------------------------------------------ indexer launch
 
 template <int HI, int DI, int QG>
-dsa_status launch_indexer_t(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
-                            const float* w, const uint8_t* k_fp8, const float* k_scale,
-                            const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
-                            int32_t rows, float* scores, int write_invalid, cudaStream_t stream,
-                            int dev) {
+dsa_status launch_indexer_t(const dsa_shape* s, const HostLayout& lay, const uint8_t* q_fp8,
+                            const float* q_scale, const float* w, const uint8_t* k_fp8,
+                            const float* k_scale, const int32_t* q_pos0, const int32_t* kv_len,
+                            int32_t row_begin, int32_t rows, float* scores, int write_invalid,
+                            cudaStream_t stream, int dev) {
   using T = dsa::IndexerTile<HI, DI, QG>;
   static std::atomic<bool> attr_done[kMaxDevices];
   if (dsa_status st = set_smem(dsa::indexer_scores_kernel<HI, DI, QG>, T::SMEM_BYTES, dev, attr_done))
@@ -210,13 +249,14 @@ dsa_status launch_indexer_t(const dsa_shape* s, const uint8_t* q_fp8, const floa
   CUtensorMap tq, tk;
   if (dsa_status st = make_tmap_u8(&tq, q_fp8, static_cast<uint64_t>(s->batch) * s->n_q * HI, DI, T::N))
     return st;
-  if (dsa_status st = make_tmap_u8(&tk, k_fp8, static_cast<uint64_t>(s->batch) * s->n_kv, DI, T::M))
+  if (dsa_status st = make_tmap_u8(&tk, k_fp8, static_cast<uint64_t>(lay.km.pool_rows), DI, T::M))
     return st;
   dsa::IndexerParams p{};
   p.q_scale = q_scale;
   p.w = w;
   p.k_scale = k_scale;
-  p.q_pos0 = q_pos0;
+  p.rp = dsa::RowPos{q_pos0, lay.row_pos, s->n_q};
+  p.km = lay.km;
   p.kv_len = kv_len;
   p.scores = scores;
   p.B = s->batch;
@@ -242,22 +282,23 @@ dsa_status launch_indexer_t(const dsa_shape* s, const uint8_t* q_fp8, const floa
   return DSA_OK;
 }
 
-dsa_status launch_indexer(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
-                          const float* w, const uint8_t* k_fp8, const float* k_scale,
-                          const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
-                          int32_t rows, float* scores, int write_invalid, cudaStream_t stream,
-                          int dev) {
+dsa_status launch_indexer(const dsa_shape* s, const HostLayout& lay, const uint8_t* q_fp8,
+                          const float* q_scale, const float* w, const uint8_t* k_fp8,
+                          const float* k_scale, const int32_t* q_pos0, const int32_t* kv_len,
+                          int32_t row_begin, int32_t rows, float* scores, int write_invalid,
+                          cudaStream_t stream, int dev) {
   if (s->idx_heads == 64) {
     if (rows == 1)
-      return launch_indexer_t<64, 128, 1>(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
-                                          row_begin, rows, scores, write_invalid, stream, dev);
-    return launch_indexer_t<64, 128, 4>(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+      return launch_indexer_t<64, 128, 1>(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0,
+                                          kv_len, row_begin, rows, scores, write_invalid, stream,
+                                          dev);
+    return launch_indexer_t<64, 128, 4>(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
                                         row_begin, rows, scores, write_invalid, stream, dev);
   }
   if (rows <= 4)
-    return launch_indexer_t<4, 32, 4>(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+    return launch_indexer_t<4, 32, 4>(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
                                       row_begin, rows, scores, write_invalid, stream, dev);
-  return launch_indexer_t<4, 32, 64>(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+  return launch_indexer_t<4, 32, 64>(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
                                      row_begin, rows, scores, write_invalid, stream, dev);
 }
 
@@ -267,11 +308,11 @@ bool indexer_topk_supported(const dsa_shape* s) {
   return s->idx_heads == 64 && s->idx_dim == 128 && s->topk <= T::MAX_K;
 }
 
-dsa_status launch_indexer_topk(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
-                               const float* w, const uint8_t* k_fp8, const float* k_scale,
-                               const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
-                               int32_t rows, int32_t* indices, int32_t out_rows,
-                               cudaStream_t stream, int dev) {
+dsa_status launch_indexer_topk(const dsa_shape* s, const HostLayout& lay, const uint8_t* q_fp8,
+                               const float* q_scale, const float* w, const uint8_t* k_fp8,
+                               const float* k_scale, const int32_t* q_pos0,
+                               const int32_t* kv_len, int32_t row_begin, int32_t rows,
+                               int32_t* indices, int32_t out_rows, cudaStream_t stream, int dev) {
   using T = dsa::IndexerTopkTile<64, 128, 4>;
   static std::atomic<bool> attr_done[kMaxDevices];
   if (dsa_status st = set_smem(dsa::indexer_topk_kernel<64, 128, 4>, T::SMEM_BYTES, dev, attr_done))
@@ -280,13 +321,14 @@ dsa_status launch_indexer_topk(const dsa_shape* s, const uint8_t* q_fp8, const f
   CUtensorMap tq, tk;
   if (dsa_status st = make_tmap_u8(&tq, q_fp8, static_cast<uint64_t>(s->batch) * s->n_q * 64, 128, T::N))
     return st;
-  if (dsa_status st = make_tmap_u8(&tk, k_fp8, static_cast<uint64_t>(s->batch) * s->n_kv, 128, T::M))
+  if (dsa_status st = make_tmap_u8(&tk, k_fp8, static_cast<uint64_t>(lay.km.pool_rows), 128, T::M))
     return st;
   dsa::IndexerTopkParams p{};
   p.q_scale = q_scale;
   p.w = w;
   p.k_scale = k_scale;
-  p.q_pos0 = q_pos0;
+  p.rp = dsa::RowPos{q_pos0, lay.row_pos, s->n_q};
+  p.km = lay.km;
   p.kv_len = kv_len;
   p.indices = indices;
   p.B = s->batch;
@@ -306,16 +348,17 @@ dsa_status launch_indexer_topk(const dsa_shape* s, const uint8_t* q_fp8, const f
 
 // ------------------------------------------------------------------ top-k launch
 
-dsa_status launch_topk(const dsa_shape* s, const float* scores, int32_t row_begin, int32_t rows,
-                       const int32_t* q_pos0, const int32_t* kv_len, int32_t* indices,
-                       int32_t out_rows, int32_t out_row0, cudaStream_t stream, int dev) {
+dsa_status launch_topk(const dsa_shape* s, const HostLayout& lay, const float* scores,
+                       int32_t row_begin, int32_t rows, const int32_t* q_pos0,
+                       const int32_t* kv_len, int32_t* indices, int32_t out_rows,
+                       int32_t out_row0, cudaStream_t stream, int dev) {
   static std::atomic<bool> attr_done[kMaxDevices];
   const int smem = static_cast<int>(sizeof(dsa::TopkSmem));
   if (dsa_status st = set_smem(dsa::topk_kernel, smem, dev, attr_done)) return st;
   if (s->batch > 65535) return fail(DSA_ERR_INVALID_ARG, "batch > 65535");
   dsa::TopkParams p{};
   p.scores = scores;
-  p.q_pos0 = q_pos0;
+  p.rp = dsa::RowPos{q_pos0, lay.row_pos, s->n_q};
   p.kv_len = kv_len;
   p.indices = indices;
   p.rows = rows;
@@ -364,9 +407,9 @@ AttnPlan plan_attn(const dsa_shape* s) {
 }
 
 template <int DQK, int DV, int VSPLIT>
-dsa_status launch_attn_t(const dsa_shape* s, const AttnPlan& pl, const uint16_t* q,
-                         const uint16_t* kv, const int32_t* indices, void* out, int out_bf16,
-                         float* lse, void* ws, cudaStream_t stream, int dev) {
+dsa_status launch_attn_t(const dsa_shape* s, const dsa::KeyMap& km, const AttnPlan& pl,
+                         const uint16_t* q, const uint16_t* kv, const int32_t* indices, void* out,
+                         int out_bf16, float* lse, void* ws, cudaStream_t stream, int dev) {
   using T = dsa::AttnTile<DQK, DV, VSPLIT>;
   static std::atomic<bool> attr_done[kMaxDevices];
   if (dsa_status st = set_smem(dsa::sparse_attn_kernel<DQK, DV, VSPLIT>, T::SMEM_BYTES, dev, attr_done))
@@ -374,6 +417,7 @@ dsa_status launch_attn_t(const dsa_shape* s, const AttnPlan& pl, const uint16_t*
   dsa::AttnParams p{};
   p.q = reinterpret_cast<const __nv_bfloat16*>(q);
   p.kv = reinterpret_cast<const __nv_bfloat16*>(kv);
+  p.km = km;
   p.indices = indices;
   p.out = out;
   p.lse = lse;
@@ -407,9 +451,10 @@ dsa_status launch_attn_t(const dsa_shape* s, const AttnPlan& pl, const uint16_t*
 }
 
 // 576/512 latent: two CTAs per (row, split), one per value half, see sparse_attn_vh.cuh.
-dsa_status launch_attn_vh(const dsa_shape* s, const AttnPlan& pl, const uint16_t* q,
-                            const uint16_t* kv, const int32_t* indices, void* out, int out_bf16,
-                            float* lse, void* ws, cudaStream_t stream, int dev) {
+dsa_status launch_attn_vh(const dsa_shape* s, const dsa::KeyMap& km, const AttnPlan& pl,
+                          const uint16_t* q, const uint16_t* kv, const int32_t* indices,
+                          void* out, int out_bf16, float* lse, void* ws, cudaStream_t stream,
+                          int dev) {
   using T = dsa::VhTile;
   static std::atomic<bool> attr_done[kMaxDevices];
   if (dsa_status st = set_smem(dsa::sparse_attn_vh_kernel, T::SMEM_BYTES, dev, attr_done))
@@ -417,6 +462,7 @@ dsa_status launch_attn_vh(const dsa_shape* s, const AttnPlan& pl, const uint16_t
   dsa::AttnParams p{};
   p.q = reinterpret_cast<const __nv_bfloat16*>(q);
   p.kv = reinterpret_cast<const __nv_bfloat16*>(kv);
+  p.km = km;
   p.indices = indices;
   p.out = out;
   p.lse = lse;
@@ -448,9 +494,9 @@ dsa_status launch_attn_vh(const dsa_shape* s, const AttnPlan& pl, const uint16_t
   return DSA_OK;
 }
 
-dsa_status launch_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv,
-                       const int32_t* indices, void* out, int out_bf16, float* lse, void* ws,
-                       size_t ws_bytes, cudaStream_t stream, int dev) {
+dsa_status launch_attn(const dsa_shape* s, const dsa::KeyMap& km, const uint16_t* q,
+                       const uint16_t* kv, const int32_t* indices, void* out, int out_bf16,
+                       float* lse, void* ws, size_t ws_bytes, cudaStream_t stream, int dev) {
   const AttnPlan pl = plan_attn(s);
   if (pl.ws_bytes > 0) {
     if (!ws || ws_bytes < pl.ws_bytes)
@@ -459,8 +505,8 @@ dsa_status launch_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv
     if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   }
   if (s->qk_dim == 576)
-    return launch_attn_vh(s, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
-  return launch_attn_t<64, 64, 1>(s, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
+    return launch_attn_vh(s, km, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
+  return launch_attn_t<64, 64, 1>(s, km, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
 }
 
 // ------------------------------------------------------------------ forward plan
@@ -635,10 +681,11 @@ dsa_status dsa_forward_plan(const dsa_shape* s, int32_t* fused, int32_t* chunk_r
   return DSA_OK;
 }
 
-dsa_status dsa_indexer_scores(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
-                              const float* w, const uint8_t* k_fp8, const float* k_scale,
-                              const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
-                              int32_t row_end, int32_t flags, float* scores, void* stream) {
+dsa_status dsa_indexer_scores_ex(const dsa_shape* s, const dsa_layout* layout,
+                                 const uint8_t* q_fp8, const float* q_scale, const float* w,
+                                 const uint8_t* k_fp8, const float* k_scale,
+                                 const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
+                                 int32_t row_end, int32_t flags, float* scores, void* stream) {
   if (dsa_status st = check_indexer_shape(s)) return st;
   if (flags != DSA_SCORES_ALL && flags != DSA_SCORES_VISIBLE_ONLY)
     return fail(DSA_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
@@ -649,17 +696,28 @@ dsa_status dsa_indexer_scores(const dsa_shape* s, const uint8_t* q_fp8, const fl
                 row_end, s->n_q);
   if (!aligned(q_fp8, 16) || !aligned(k_fp8, 16))
     return fail(DSA_ERR_INVALID_ARG, "q_fp8 and k_fp8 must be 16-byte aligned");
+  HostLayout lay;
+  if (dsa_status st = resolve_layout(s, layout, &lay)) return st;
   int dev;
   if (dsa_status st = current_device(&dev)) return st;
-  return launch_indexer(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, row_begin,
+  return launch_indexer(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, row_begin,
                         row_end - row_begin, scores, flags == DSA_SCORES_ALL ? 1 : 0,
                         static_cast<cudaStream_t>(stream), dev);
 }
 
-dsa_status dsa_indexer_topk(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
-                            const float* w, const uint8_t* k_fp8, const float* k_scale,
-                            const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
-                            int32_t row_end, int32_t* indices, void* stream) {
+dsa_status dsa_indexer_scores(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
+                              const float* w, const uint8_t* k_fp8, const float* k_scale,
+                              const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
+                              int32_t row_end, int32_t flags, float* scores, void* stream) {
+  return dsa_indexer_scores_ex(s, nullptr, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+                               row_begin, row_end, flags, scores, stream);
+}
+
+dsa_status dsa_indexer_topk_ex(const dsa_shape* s, const dsa_layout* layout, const uint8_t* q_fp8,
+                               const float* q_scale, const float* w, const uint8_t* k_fp8,
+                               const float* k_scale, const int32_t* q_pos0,
+                               const int32_t* kv_len, int32_t row_begin, int32_t row_end,
+                               int32_t* indices, void* stream) {
   if (dsa_status st = check_indexer_shape(s)) return st;
   if (dsa_status st = check_topk_shape(s)) return st;
   if (!indexer_topk_supported(s))
@@ -674,16 +732,27 @@ dsa_status dsa_indexer_topk(const dsa_shape* s, const uint8_t* q_fp8, const floa
                 row_end, s->n_q);
   if (!aligned(q_fp8, 16) || !aligned(k_fp8, 16))
     return fail(DSA_ERR_INVALID_ARG, "q_fp8 and k_fp8 must be 16-byte aligned");
+  HostLayout lay;
+  if (dsa_status st = resolve_layout(s, layout, &lay)) return st;
   int dev;
   if (dsa_status st = current_device(&dev)) return st;
-  return launch_indexer_topk(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, row_begin,
+  return launch_indexer_topk(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, row_begin,
                              row_end - row_begin, indices, row_end - row_begin,
                              static_cast<cudaStream_t>(stream), dev);
 }
 
-dsa_status dsa_topk(const dsa_shape* s, const float* scores, int32_t row_begin, int32_t row_end,
-                    const int32_t* q_pos0, const int32_t* kv_len, int32_t* indices, void* ws,
-                    size_t ws_bytes, void* stream) {
+dsa_status dsa_indexer_topk(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
+                            const float* w, const uint8_t* k_fp8, const float* k_scale,
+                            const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
+                            int32_t row_end, int32_t* indices, void* stream) {
+  return dsa_indexer_topk_ex(s, nullptr, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+                             row_begin, row_end, indices, stream);
+}
+
+dsa_status dsa_topk_ex(const dsa_shape* s, const dsa_layout* layout, const float* scores,
+                       int32_t row_begin, int32_t row_end, const int32_t* q_pos0,
+                       const int32_t* kv_len, int32_t* indices, void* ws, size_t ws_bytes,
+                       void* stream) {
   (void)ws;
   (void)ws_bytes;
   if (dsa_status st = check_topk_shape(s)) return st;
@@ -691,25 +760,43 @@ dsa_status dsa_topk(const dsa_shape* s, const float* scores, int32_t row_begin, 
   if (row_begin < 0 || row_end > s->n_q || row_begin >= row_end)
     return fail(DSA_ERR_INVALID_ARG, "row range [%d, %d) outside [0, %d) or empty", row_begin,
                 row_end, s->n_q);
+  HostLayout lay;
+  if (dsa_status st = resolve_layout(s, layout, &lay)) return st;
   int dev;
   if (dsa_status st = current_device(&dev)) return st;
-  return launch_topk(s, scores, row_begin, row_end - row_begin, q_pos0, kv_len, indices,
+  return launch_topk(s, lay, scores, row_begin, row_end - row_begin, q_pos0, kv_len, indices,
                      row_end - row_begin, 0, static_cast<cudaStream_t>(stream), dev);
 }
 
-dsa_status dsa_sparse_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv,
-                           const int32_t* indices, void* out, int32_t out_dtype, float* lse,
-                           void* ws, size_t ws_bytes, void* stream) {
+dsa_status dsa_topk(const dsa_shape* s, const float* scores, int32_t row_begin, int32_t row_end,
+                    const int32_t* q_pos0, const int32_t* kv_len, int32_t* indices, void* ws,
+                    size_t ws_bytes, void* stream) {
+  return dsa_topk_ex(s, nullptr, scores, row_begin, row_end, q_pos0, kv_len, indices, ws,
+                     ws_bytes, stream);
+}
+
+dsa_status dsa_sparse_attn_ex(const dsa_shape* s, const dsa_layout* layout, const uint16_t* q,
+                              const uint16_t* kv, const int32_t* indices, void* out,
+                              int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+                              void* stream) {
   if (dsa_status st = check_attn_shape(s)) return st;
   if (dsa_status st = check_ptrs({q, kv, indices, out}, "dsa_sparse_attn")) return st;
   if (out_dtype != DSA_OUT_F32 && out_dtype != DSA_OUT_BF16)
     return fail(DSA_ERR_INVALID_ARG, "out_dtype must be DSA_OUT_F32 or DSA_OUT_BF16");
   if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(out, 16))
     return fail(DSA_ERR_INVALID_ARG, "q, kv and out must be 16-byte aligned");
+  HostLayout lay;
+  if (dsa_status st = resolve_layout(s, layout, &lay)) return st;
   int dev;
   if (dsa_status st = current_device(&dev)) return st;
-  return launch_attn(s, q, kv, indices, out, out_dtype == DSA_OUT_BF16, lse, ws, ws_bytes,
+  return launch_attn(s, lay.km, q, kv, indices, out, out_dtype == DSA_OUT_BF16, lse, ws, ws_bytes,
                      static_cast<cudaStream_t>(stream), dev);
+}
+
+dsa_status dsa_sparse_attn(const dsa_shape* s, const uint16_t* q, const uint16_t* kv,
+                           const int32_t* indices, void* out, int32_t out_dtype, float* lse,
+                           void* ws, size_t ws_bytes, void* stream) {
+  return dsa_sparse_attn_ex(s, nullptr, q, kv, indices, out, out_dtype, lse, ws, ws_bytes, stream);
 }
 
 dsa_status dsa_sparse_attn_noalloc(const dsa_shape* s, const uint16_t* q, const uint16_t* kv,
@@ -727,22 +814,25 @@ dsa_status dsa_sparse_attn_noalloc(const dsa_shape* s, const uint16_t* q, const 
                 "this shape needs %zu bytes of split-K scratch; dsa_sparse_attn_noalloc holds at "
                 "most %zu (use dsa_sparse_attn with a workspace)",
                 pl.ws_bytes, kNoAllocScratchBytes);
+  HostLayout lay;
+  if (dsa_status st = resolve_layout(s, nullptr, &lay)) return st;
   int dev;
   if (dsa_status st = current_device(&dev)) return st;
   void* scratch = nullptr;
   if (pl.ws_bytes > 0) {
     if (dsa_status st = noalloc_scratch_addr(dev, &scratch)) return st;
   }
-  return launch_attn(s, q, kv, indices, out, out_dtype == DSA_OUT_BF16, lse, scratch,
+  return launch_attn(s, lay.km, q, kv, indices, out, out_dtype == DSA_OUT_BF16, lse, scratch,
                      pl.ws_bytes > 0 ? kNoAllocScratchBytes : 0,
                      static_cast<cudaStream_t>(stream), dev);
 }
 
-dsa_status dsa_forward(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
-                       const float* w, const uint8_t* k_fp8, const float* k_scale,
-                       const int32_t* q_pos0, const int32_t* kv_len, const uint16_t* q,
-                       const uint16_t* kv, int32_t* indices_out, void* out, int32_t out_dtype,
-                       float* lse, void* ws, size_t ws_bytes, void* stream) {
+dsa_status dsa_forward_ex(const dsa_shape* s, const dsa_layout* layout, const uint8_t* q_fp8,
+                          const float* q_scale, const float* w, const uint8_t* k_fp8,
+                          const float* k_scale, const int32_t* q_pos0, const int32_t* kv_len,
+                          const uint16_t* q, const uint16_t* kv, int32_t* indices_out, void* out,
+                          int32_t out_dtype, float* lse, void* ws, size_t ws_bytes,
+                          void* stream) {
   if (dsa_status st = check_indexer_shape(s)) return st;
   if (dsa_status st = check_attn_shape(s)) return st;
   if (dsa_status st = check_ptrs({q_fp8, q_scale, w, k_fp8, k_scale, q, kv, indices_out, out},
@@ -753,6 +843,8 @@ dsa_status dsa_forward(const dsa_shape* s, const uint8_t* q_fp8, const float* q_
   if (!aligned(q_fp8, 16) || !aligned(k_fp8, 16) || !aligned(q, 16) || !aligned(kv, 16) ||
       !aligned(out, 16))
     return fail(DSA_ERR_INVALID_ARG, "q_fp8, k_fp8, q, kv and out must be 16-byte aligned");
+  HostLayout lay;
+  if (dsa_status st = resolve_layout(s, layout, &lay)) return st;
   const FwdPlan f = plan_forward(s);
   if (f.total > 0) {
     if (!ws || ws_bytes < f.total)
@@ -766,24 +858,33 @@ dsa_status dsa_forward(const dsa_shape* s, const uint8_t* q_fp8, const float* q_
   float* scores = static_cast<float*>(ws);
   void* attn_ws = static_cast<char*>(ws) + f.scores_bytes;
   if (f.fused) {
-    if (dsa_status e = launch_indexer_topk(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
-                                           0, s->n_q, indices_out, s->n_q, st_, dev))
+    if (dsa_status e = launch_indexer_topk(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0,
+                                           kv_len, 0, s->n_q, indices_out, s->n_q, st_, dev))
       return e;
-    return launch_attn(s, q, kv, indices_out, out, out_dtype == DSA_OUT_BF16, lse, attn_ws,
+    return launch_attn(s, lay.km, q, kv, indices_out, out, out_dtype == DSA_OUT_BF16, lse, attn_ws,
                        f.attn_bytes, st_, dev);
   }
   for (int r0 = 0; r0 < s->n_q; r0 += f.chunk_rows) {
     const int rows = std::min(f.chunk_rows, s->n_q - r0);
-    if (dsa_status e = launch_indexer(s, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, r0,
-                                      rows, scores, 0, st_, dev))
+    if (dsa_status e = launch_indexer(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+                                      r0, rows, scores, 0, st_, dev))
       return e;
     // The chunk's selections go straight to their rows of indices_out.
-    if (dsa_status e = launch_topk(s, scores, r0, rows, q_pos0, kv_len, indices_out, s->n_q, r0,
-                                   st_, dev))
+    if (dsa_status e = launch_topk(s, lay, scores, r0, rows, q_pos0, kv_len, indices_out, s->n_q,
+                                   r0, st_, dev))
       return e;
   }
-  return launch_attn(s, q, kv, indices_out, out, out_dtype == DSA_OUT_BF16, lse, attn_ws,
+  return launch_attn(s, lay.km, q, kv, indices_out, out, out_dtype == DSA_OUT_BF16, lse, attn_ws,
                      f.attn_bytes, st_, dev);
+}
+
+dsa_status dsa_forward(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
+                       const float* w, const uint8_t* k_fp8, const float* k_scale,
+                       const int32_t* q_pos0, const int32_t* kv_len, const uint16_t* q,
+                       const uint16_t* kv, int32_t* indices_out, void* out, int32_t out_dtype,
+                       float* lse, void* ws, size_t ws_bytes, void* stream) {
+  return dsa_forward_ex(s, nullptr, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, q, kv,
+                        indices_out, out, out_dtype, lse, ws, ws_bytes, stream);
 }
 
 dsa_status dsa_check(void* stream) {
@@ -799,6 +900,11 @@ dsa_status dsa_check(void* stream) {
       return fail(DSA_ERR_TIMEOUT, "a device-side wait exceeded its limit (error word 0x%x)", word);
     if (word & dsa::kErrInternal)
       return fail(DSA_ERR_CUDA, "a kernel invariant failed (error word 0x%x)", word);
+    if (word & dsa::kErrBadInput)
+      return fail(DSA_ERR_INVALID_ARG,
+                  "a block-table page was outside the key pool; its keys were skipped "
+                  "(error word 0x%x)",
+                  word);
     return fail(DSA_ERR_CUDA, "device error word 0x%x", word);
   }
   return DSA_OK;

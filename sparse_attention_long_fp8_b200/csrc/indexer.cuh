@@ -18,6 +18,7 @@
 // accumulators), warps 2.. run the epilogue.
 #pragma once
 
+#include "layout.cuh"
 #include "ptx.cuh"
 
 namespace dsa {
@@ -25,8 +26,9 @@ namespace dsa {
 struct IndexerParams {
   const float* q_scale;   // [B, n_q, HI]
   const float* w;         // [B, n_q, HI]
-  const float* k_scale;   // [B, n_kv]
-  const int32_t* q_pos0;  // [B] or null
+  const float* k_scale;   // [pool rows] (contiguous: [B, n_kv])
+  RowPos rp;              // absolute position of each query row
+  KeyMap km;              // pool row of each key
   const int32_t* kv_len;  // [B] or null
   float* scores;          // [B, rows, n_kv]
   int32_t B, n_q, n_kv;
@@ -89,9 +91,10 @@ __global__ void __launch_bounds__(IndexerTile<HI, DI, QG>::THREADS, 1)
 
   const int r0 = p.row_begin + group * QG;                   // first row of the group
   const int r_last = min(r0 + QG, p.row_begin + p.rows) - 1;  // last row scored here
-  const int pos0 = p.q_pos0 ? p.q_pos0[b] : 0;
   const int kvl = min(p.kv_len ? p.kv_len[b] : p.n_kv, p.n_kv);
-  const int key_end = max(0, min(kvl, pos0 + r_last + 1));   // visible keys of the group
+  int pos_max = -1;                                          // latest position in the group
+  for (int r = r0; r <= r_last; ++r) pos_max = max(pos_max, p.rp.pos(b, r));
+  const int key_end = max(0, min(kvl, pos_max + 1));         // visible keys of the group
   const int n_tiles_all = (p.n_kv + T::M - 1) / T::M;
   const int t_begin = split * p.tiles_per_split;
   const int t_end = min(t_begin + p.tiles_per_split, n_tiles_all);
@@ -143,8 +146,10 @@ __global__ void __launch_bounds__(IndexerTile<HI, DI, QG>::THREADS, 1)
         const int st = i % T::STAGES;
         if (!mbar_wait(&k_empty[st], ((i / T::STAGES) & 1) ^ 1)) break;
         mbar_arrive_expect_tx(&k_full[st], T::K_BYTES);
+        // a page outside the pool reads the TMA fill (zeros) past its end
+        const int64_t y = p.km.row(b, (t_begin + i) * T::M, p.n_kv);
         tma_load_2d(k_smem + st * T::K_BYTES, &tmap_k, &k_full[st], 0,
-                    b * p.n_kv + (t_begin + i) * T::M);
+                    static_cast<int32_t>(y >= 0 ? y : p.km.pool_rows));
         ++issued;
       }
       // Drain: every issued key tile has landed before the CTA may exit.
@@ -188,17 +193,23 @@ __global__ void __launch_bounds__(IndexerTile<HI, DI, QG>::THREADS, 1)
     float* out_base = p.scores + (static_cast<size_t>(b) * p.rows + (r0 - p.row_begin)) * row_stride;
 
     float cf[T::QPW][HI];
+    int rpos[T::QPW];
 #pragma unroll
-    for (int q = 0; q < T::QPW; ++q)
+    for (int q = 0; q < T::QPW; ++q) {
+      const int r = r0 + qhalf * T::QPW + q;
+      rpos[q] = r <= r_last ? p.rp.pos(b, r) : -1;
 #pragma unroll
       for (int j = 0; j < HI; ++j) cf[q][j] = coef[(qhalf * T::QPW + q) * HI + j];
+    }
 
     // The key scale of tile i + 1 is loaded while tile i is processed, so its
-    // global-memory latency is not on the per-tile path.
-    const float* ks_row = p.k_scale + static_cast<size_t>(b) * p.n_kv;
+    // global-memory latency is not on the per-tile path. A tile lies inside
+    // one page, so its first key's pool row locates all of its keys.
     auto load_ks = [&](int i) -> float {
-      const int s = (t_begin + i) * T::M + key_local;
-      return (i < n_compute && s < p.n_kv) ? ks_row[s] : 0.f;
+      const int s0 = (t_begin + i) * T::M;
+      if (i >= n_compute || s0 + key_local >= p.n_kv) return 0.f;
+      const int64_t r = p.km.row(b, s0, p.n_kv);
+      return r >= 0 ? p.k_scale[r + key_local] : 0.f;
     };
     float ks_next = load_ks(0);
     bool ok = true;
@@ -235,7 +246,7 @@ __global__ void __launch_bounds__(IndexerTile<HI, DI, QG>::THREADS, 1)
         }
         const int r = r0 + ql;
         if (r <= r_last && s < p.n_kv) {
-          const bool vis = s <= pos0 + r && s < kvl;
+          const bool vis = s <= rpos[q] && s < kvl;
           out_base[static_cast<size_t>(ql) * row_stride + s] = vis ? acc * ks : -INFINITY;
         }
       }

@@ -33,6 +33,7 @@
 // (one TMEM lane quarter each).
 #pragma once
 
+#include "layout.cuh"
 #include "ptx.cuh"
 
 namespace dsa {
@@ -40,8 +41,9 @@ namespace dsa {
 struct IndexerTopkParams {
   const float* q_scale;   // [B, n_q, HI]
   const float* w;         // [B, n_q, HI]
-  const float* k_scale;   // [B, n_kv]
-  const int32_t* q_pos0;  // [B] or null
+  const float* k_scale;   // [pool rows] (contiguous: [B, n_kv])
+  RowPos rp;              // absolute position of each query row
+  KeyMap km;              // pool row of each key
   const int32_t* kv_len;  // [B] or null
   int32_t* indices;       // row r of sequence b -> indices[(b * out_rows + r - row_begin) * k]
   int32_t B, n_q, n_kv, k;
@@ -451,9 +453,10 @@ __global__ void __launch_bounds__(IndexerTopkTile<HI, DI, QG>::THREADS, 1)
 
   const int r0 = p.row_begin + group * QG;                   // first row of the group
   const int r_last = min(r0 + QG, p.row_begin + p.rows) - 1;  // last row selected here
-  const int pos0 = p.q_pos0 ? p.q_pos0[b] : 0;
   const int kvl = min(p.kv_len ? p.kv_len[b] : p.n_kv, p.n_kv);
-  const int key_end = max(0, min(kvl, pos0 + r_last + 1));   // visible keys of the group
+  int pos_max = -1;                                          // latest position in the group
+  for (int r = r0; r <= r_last; ++r) pos_max = max(pos_max, p.rp.pos(b, r));
+  const int key_end = max(0, min(kvl, pos_max + 1));         // visible keys of the group
   const int n_compute = (key_end + T::M - 1) / T::M;
 
   if (threadIdx.x == 0) {
@@ -507,7 +510,10 @@ __global__ void __launch_bounds__(IndexerTopkTile<HI, DI, QG>::THREADS, 1)
         const int st = i % T::STAGES;
         if (!mbar_wait(&k_empty[st], ((i / T::STAGES) & 1) ^ 1)) break;
         mbar_arrive_expect_tx(&k_full[st], T::K_BYTES);
-        tma_load_2d(k_smem + st * T::K_BYTES, &tmap_k, &k_full[st], 0, b * p.n_kv + i * T::M);
+        // a page outside the pool reads the TMA fill (zeros) past its end
+        const int64_t y = p.km.row(b, i * T::M, p.n_kv);
+        tma_load_2d(k_smem + st * T::K_BYTES, &tmap_k, &k_full[st], 0,
+                    static_cast<int32_t>(y >= 0 ? y : p.km.pool_rows));
         ++issued;
       }
       // Drain: every issued key tile has landed before the CTA may exit.
@@ -572,11 +578,20 @@ __global__ void __launch_bounds__(IndexerTopkTile<HI, DI, QG>::THREADS, 1)
     // so that the group's barriers stay matched.
     // The key scale of tile i + 1 is loaded while tile i is processed, so its
     // global-memory latency is not on the per-tile path.
-    const float* ks_row = p.k_scale + static_cast<size_t>(b) * p.n_kv;
+    // A tile lies inside one page, so its first key's pool row locates all
+    // of its keys.
     auto load_ks = [&](int i) -> float {
-      const int s = i * T::M + key_local;
-      return (i < n_compute && s < p.n_kv) ? ks_row[s] : 0.f;
+      const int s0 = i * T::M;
+      if (i >= n_compute || s0 + key_local >= p.n_kv) return 0.f;
+      const int64_t r = p.km.row(b, s0, p.n_kv);
+      return r >= 0 ? p.k_scale[r + key_local] : 0.f;
     };
+    int rpos[T::QPW];
+#pragma unroll
+    for (int q = 0; q < T::QPW; ++q) {
+      const int r = r0 + qhalf * T::QPW + q;
+      rpos[q] = r <= r_last ? p.rp.pos(b, r) : -1;
+    }
     float ks_next = load_ks(0);
     bool ok = true;
     for (int i = 0; i < n_compute; ++i) {
@@ -609,7 +624,7 @@ __global__ void __launch_bounds__(IndexerTopkTile<HI, DI, QG>::THREADS, 1)
           acc = fmaf(__uint_as_float(c4.w), fmaxf(__uint_as_float(x[q][j + 3]), 0.f), acc);
         }
         const int r = r0 + ql;
-        const bool vis = r <= r_last && s < p.n_kv && s <= pos0 + r && s < kvl;
+        const bool vis = r <= r_last && s < p.n_kv && s <= rpos[q] && s < kvl;
         const uint32_t u = score_key(acc * ks);
         // A key equal to tau with an index above tau_idx loses the tie to the
         // k kept entries (keys arrive in increasing index order).

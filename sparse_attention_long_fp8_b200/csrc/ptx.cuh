@@ -17,6 +17,9 @@ __device__ unsigned int g_error_word;
 constexpr unsigned int kErrTimeout = 1u;
 // A kernel found one of its own invariants broken (a bug, never an input error).
 constexpr unsigned int kErrInternal = 2u;
+// A device-side input was out of range (a block-table page outside the pool);
+// the access was skipped.
+constexpr unsigned int kErrBadInput = 4u;
 // Bounded waits give up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 

@@ -26,13 +26,15 @@
 
 #include <cuda_bf16.h>
 
+#include "layout.cuh"
 #include "ptx.cuh"
 
 namespace dsa {
 
 struct AttnParams {
   const __nv_bfloat16* q;   // [B, n_q, H, DQK]
-  const __nv_bfloat16* kv;  // [B, n_kv, DQK]
+  const __nv_bfloat16* kv;  // [pool rows, DQK] latent rows (contiguous: [B, n_kv, DQK])
+  KeyMap km;                // pool row of each key
   const int32_t* indices;   // [B, n_q, topk]
   void* out;                // [B, n_q, H, DV] fp32 or bf16
   float* lse;               // [B, n_q, H] or null
@@ -100,7 +102,6 @@ __global__ void __launch_bounds__(288, 1)
   const int slot_end = min(p.topk, slot_begin + p.slots_per_split);
   const int n_blocks = max(0, (slot_end - slot_begin + NK - 1) / NK);
   const int32_t* row_idx = p.indices + static_cast<size_t>(row) * p.topk;
-  const __nv_bfloat16* kv_b = p.kv + static_cast<size_t>(b) * p.n_kv * DQK;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, T::PRODUCERS);
@@ -154,9 +155,10 @@ __global__ void __launch_bounds__(288, 1)
         const int db = rem >> 3, ch = rem & 7;
         const int slot = slot0 + j;
         const int idx = slot < slot_end ? row_idx[slot] : -1;
-        const bool valid = idx >= 0 && idx < p.n_kv;
+        const int64_t krow = (idx >= 0 && idx < p.n_kv) ? p.km.row(b, idx, p.n_kv) : -1;
+        const bool valid = krow >= 0;
         const uint32_t dst = c_addr + db * (NK * 128) + j * 128 + ((ch ^ (j & 7)) << 4);
-        const void* src = valid ? static_cast<const void*>(kv_b + static_cast<size_t>(idx) * DQK + db * 64 + ch * 8)
+        const void* src = valid ? static_cast<const void*>(p.kv + krow * DQK + db * 64 + ch * 8)
                                 : static_cast<const void*>(p.kv);
         cp_async_16(dst, src, valid ? 16u : 0u);
       }

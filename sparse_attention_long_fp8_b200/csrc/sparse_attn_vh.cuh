@@ -116,7 +116,6 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
   const int slot_end = min(p.topk, slot_begin + p.slots_per_split);
   const int n_blocks = max(0, (slot_end - slot_begin + NK - 1) / NK);
   const int32_t* row_idx = p.indices + static_cast<size_t>(row) * p.topk;
-  const __nv_bfloat16* kv_b = p.kv + static_cast<size_t>(b) * p.n_kv * T::DQK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < T::STAGES; ++s) {
@@ -154,12 +153,12 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
     // instruction moves four whole 128-byte lines.
     const int kq = threadIdx.x >> 3, ch = threadIdx.x & 7;
     const uint32_t dst0 = smem_u32(c_smem) + kq * 128 + ((ch ^ (kq & 7)) << 4);
-    auto load_keys = [&](int blk, int (&k)[4]) {
+    auto load_keys = [&](int blk, int64_t (&k)[4]) {
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int slot = slot_begin + blk * NK + kq + 16 * r;
         const int idx = (blk < n_blocks && slot < slot_end) ? row_idx[slot] : -1;
-        k[r] = (idx >= 0 && idx < p.n_kv) ? idx : -1;
+        k[r] = (idx >= 0 && idx < p.n_kv) ? p.km.row(b, idx, p.n_kv) : -1;   // pool row
       }
     };
     auto copy_part = [&](auto vh_c, auto vpart_c, uint32_t dst, const __nv_bfloat16* const (&src)[4],
@@ -178,7 +177,7 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
     using I1 = std::integral_constant<int, 1>;
     using BX = std::integral_constant<bool, false>;
     using BV = std::integral_constant<bool, true>;
-    int keys[4];
+    int64_t keys[4];
     load_keys(0, keys);
     bool ok = true;
     for (int i = 0; i < n_blocks && ok; ++i) {
@@ -188,7 +187,7 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
       uint32_t bytes[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        src[r] = kv_b + static_cast<size_t>(keys[r] >= 0 ? keys[r] : 0) * T::DQK + ch * 8;
+        src[r] = p.kv + (keys[r] >= 0 ? keys[r] : 0) * T::DQK + ch * 8;
         bytes[r] = keys[r] >= 0 ? 16u : 0u;
       }
       load_keys(i + 1, keys);   // one block ahead

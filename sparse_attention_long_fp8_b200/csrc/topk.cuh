@@ -18,13 +18,14 @@
 // row the exact select has to look at.
 #pragma once
 
+#include "layout.cuh"
 #include "ptx.cuh"
 
 namespace dsa {
 
 struct TopkParams {
   const float* scores;    // [B, rows, n_kv]
-  const int32_t* q_pos0;  // [B] or null
+  RowPos rp;              // absolute position of each query row
   const int32_t* kv_len;  // [B] or null
   int32_t* indices;       // row r of sequence b -> indices[(b * out_rows + out_row0 + r) * k]
   int32_t rows, row_begin, n_kv, k;   // score rows [row_begin, row_begin + rows) per sequence
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
 
   const int r = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const int pos = (p.q_pos0 ? p.q_pos0[b] : 0) + p.row_begin + r;
+  const int pos = p.rp.pos(b, p.row_begin + r);
   const int kvl = min(p.kv_len ? p.kv_len[b] : p.n_kv, p.n_kv);
   const int n = max(0, min(pos + 1, kvl));
   const float* row = p.scores + (static_cast<size_t>(b) * p.rows + r) * p.n_kv;

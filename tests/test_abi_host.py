@@ -171,3 +171,44 @@ def test_valid_call_without_device_reports_no_device(lib):
         pytest.skip("a GPU is present")
     st = _call_indexer(lib, _shape())
     assert st == dsa.DSA_ERR_NO_DEVICE
+
+
+def _layout(page, max_pages, pool_rows, table=FAKE, row_pos=None):
+    lay = dsa.DsaLayout()
+    lay.row_pos = row_pos
+    lay.block_table = table
+    lay.max_pages = max_pages
+    lay.page_size = page
+    lay.pool_rows = pool_rows
+    return lay
+
+
+@pytest.mark.parametrize("page,max_pages,pool_rows,table", [
+    (100, 64, 64 * 100, FAKE),          # not a power of two
+    (64, 128, 64 * 128, FAKE),          # below one indexer tile
+    (256, 15, 256 * 64, FAKE),          # 4096 keys need 16 pages
+    (256, 16, 256 * 64 + 3, FAKE),      # pool not a whole number of pages
+    (256, 16, 1 << 31, FAKE),           # pool past the 32-bit TMA coordinate
+    (256, 16, 256 * 64, FAKE + 2),      # misaligned table
+])
+def test_paged_layout_checks_before_launch(lib, page, max_pages, pool_rows, table):
+    lay = _layout(page, max_pages, pool_rows, table)
+    st = lib.dsa_forward_ex(ctypes.byref(_shape()), ctypes.byref(lay), FAKE, FAKE, FAKE, FAKE,
+                            FAKE, None, None, FAKE, FAKE, FAKE, FAKE, 0, None, None, 0, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+    st = lib.dsa_sparse_attn_ex(ctypes.byref(_shape()), ctypes.byref(lay), FAKE, FAKE, FAKE, FAKE,
+                                0, None, None, 0, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_row_pos_alignment_checked(lib):
+    lay = _layout(0, 0, 0, table=None, row_pos=FAKE + 2)
+    st = lib.dsa_indexer_scores_ex(ctypes.byref(_shape()), ctypes.byref(lay), FAKE, FAKE, FAKE,
+                                   FAKE, FAKE, None, None, 0, 16, 0, FAKE, None)
+    assert st == dsa.DSA_ERR_INVALID_ARG
+
+
+def test_forward_plan_query(lib):
+    assert dsa.forward_plan(_shape()) == {"fused": True, "chunk_rows": 4096, "attn_splits": 1}
+    dec = dsa.forward_plan(dsa.shape_of(dsa.CONFIGS["decode_32k"]))
+    assert dec["fused"] is False and dec["chunk_rows"] == 1
