@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--shard", action="store_true",
+                    help="run the query-sharded prefill path even on one rank")
     return ap.parse_args()
 
 
@@ -171,11 +173,31 @@ class Step:
     step) and the same launches through the stage calls (the per-kernel
     breakdown), following the plan dsa_forward_plan reports."""
 
-    def __init__(self, cfg, seed, device):
+    def __init__(self, cfg, seed, device, dist=None, shard=None):
+        """shard = (rank, ranks): this rank's 4-row query groups of the one
+        prefill all ranks share (same seed everywhere), with the keys held
+        sequence-sharded and all-gathered each step; None: the whole
+        workload on this GPU."""
         import torch
         import sparse_attention_long_fp8_b200 as dsa
-        self.dsa, self.torch, self.cfg = dsa, torch, cfg
-        self.inp = dsa.make_inputs(cfg, seed=seed, device=device)
+        from sparse_attention_long_fp8_b200 import inputs, shard as shard_mod
+        self.dsa, self.torch, self.dist = dsa, torch, dist
+        self.full_cfg = cfg
+        inp = dsa.make_inputs(cfg, seed=seed, device=device)
+        self.layout, self.key_local = None, None
+        if shard is not None:
+            rank, ranks = shard
+            rows = shard_mod.shard_rows(cfg.n_q, ranks, rank)
+            inp = shard_mod.shard_inputs(inp, rows)
+            cfg = inputs.custom_config(cfg.name, n_q=len(rows), name=f"{cfg.name}_shard{rank}")
+            self.layout = dsa.make_layout(row_pos=inp["row_pos"])
+            if dist is not None:
+                # this rank's slice of the keys; the full tensors are refilled
+                # by the all-gather of every step
+                k0, k1 = shard_mod.key_slice(cfg.n_kv, ranks, rank)
+                self.key_local = {k: inp[k][:, k0:k1].clone() for k in ("k_fp8", "k_scale", "kv")}
+        self.cfg, self.inp = cfg, inp
+        self.shard_mod = shard_mod
         self.shape = dsa.shape_of(cfg)
         B, T = cfg.batch, cfg.n_q
         plan = dsa.forward_plan(self.shape)
@@ -195,12 +217,22 @@ class Step:
         per_chunk = 1 if self.fused else 2
         self.launches = per_chunk * len(self.chunks) + 1 + (1 if self.attn_splits > 1 else 0)
 
+    def gather_keys(self):
+        """Sharded prefill: every rank's key slices into this GPU's full key
+        tensors (NCCL all-gather)."""
+        if self.key_local is None:
+            return
+        for k, loc in self.key_local.items():
+            self.inp[k].copy_(self.shard_mod.all_gather_keys(loc, self.cfg.n_kv, self.dist))
+
     def run_forward(self):
         """One step through the public call."""
+        self.gather_keys()
         x = self.inp
         self.dsa.dsa_forward(self.shape, x["q_fp8"], x["q_scale"], x["w"], x["k_fp8"],
                              x["k_scale"], x["q_pos0"], x["kv_len"], x["q"], x["kv"], self.idx,
-                             self.out, self.lse, self.fwd_ws, self.fwd_ws_bytes)
+                             self.out, self.lse, self.fwd_ws, self.fwd_ws_bytes,
+                             layout=self.layout)
 
     def run(self, ev=None):
         """The same launches through the stage calls; with ev (a dict of event
@@ -209,24 +241,30 @@ class Step:
         dsa, x, cfg = self.dsa, self.inp, self.cfg
         rec = (lambda name: ev[name].append(self.torch.cuda.Event(enable_timing=True)) or
                ev[name][-1].record()) if ev is not None else (lambda name: None)
+        lay = self.layout
+        if self.key_local is not None:
+            rec("gather")
+            self.gather_keys()
+            rec("gather")
         if self.fused:
             rec("indexer")
             dsa.dsa_indexer_topk(self.shape, x["q_fp8"], x["q_scale"], x["w"], x["k_fp8"],
-                                 x["k_scale"], x["q_pos0"], x["kv_len"], 0, cfg.n_q, self.idx)
+                                 x["k_scale"], x["q_pos0"], x["kv_len"], 0, cfg.n_q, self.idx,
+                                 layout=lay)
             rec("indexer")
         for r0, r1 in ([] if self.fused else self.chunks):
             rec("indexer")
             dsa.dsa_indexer_scores(self.shape, x["q_fp8"], x["q_scale"], x["w"], x["k_fp8"],
                                    x["k_scale"], x["q_pos0"], x["kv_len"], r0, r1, self.scores,
-                                   flags=dsa.DSA_SCORES_VISIBLE_ONLY)
+                                   flags=dsa.DSA_SCORES_VISIBLE_ONLY, layout=lay)
             rec("indexer")
             rec("topk")
             dsa.dsa_topk(self.shape, self.scores, r0, r1, x["q_pos0"], x["kv_len"],
-                         self.idx[:, r0:r1] if cfg.batch == 1 else self.idx)
+                         self.idx[:, r0:r1] if cfg.batch == 1 else self.idx, layout=lay)
             rec("topk")
         rec("attn")
         dsa.dsa_sparse_attn(self.shape, x["q"], x["kv"], self.idx, self.out, self.lse,
-                            self.attn_ws, self.attn_ws_bytes)
+                            self.attn_ws, self.attn_ws_bytes, layout=lay)
         rec("attn")
 
 
@@ -343,7 +381,7 @@ def breakdown(step, steps):
     """K eager steps through the stage calls, each launch between CUDA events
     on the launching stream: per-kernel times for the rooflines."""
     import torch
-    ev = {"indexer": [], "topk": [], "attn": []}
+    ev = {"gather": [], "indexer": [], "topk": [], "attn": []}
     step.run()
     torch.cuda.synchronize()
     for _ in range(steps):
@@ -378,27 +416,40 @@ def attn_traffic(cfg):
     return cap["bytes"] / cap["rows"] * cfg.batch * cfg.n_q
 
 
-def prefill_leg(cfg, seed, steps, warmup, dist, peaks):
+def prefill_leg(cfg, seed, steps, warmup, dist, peaks, shard=None):
     """dsa_forward over one prefill workload: tokens/s from the timed calls,
-    per-kernel TFLOP/s from the breakdown pass."""
+    per-kernel TFLOP/s from the breakdown pass. With shard = (rank, ranks)
+    this rank runs its share of the one prefill all ranks split; the flop
+    rates are then this rank's share of the work over its kernel times."""
     import torch
-    step = Step(cfg, seed, "cuda")
+    step = Step(cfg, seed, "cuda", dist=dist, shard=shard)
     log(f"[bench] {cfg.name}: fused {step.fused}, chunk rows {step.chunk}, "
         f"{step.launches} launches/step")
     ms = timed(step, steps, warmup, dist)
     stages = breakdown(step, steps)
     launches = step.launches
     fused = step.fused
+    rows = step.cfg.n_q
+    if shard is not None:
+        from sparse_attention_long_fp8_b200 import shard as shard_mod
+        vis, sel = shard_mod.shard_cost(cfg.n_q, cfg.n_kv, shard[1], shard[0], cfg.topk)
+        ix_f = 2.0 * cfg.idx_heads * cfg.idx_dim * vis
+        at_f = 2.0 * cfg.heads * (cfg.qk_dim + cfg.v_dim) * sel
+    else:
+        ix_f, at_f = indexer_flops(cfg), attn_flops(cfg)
     del step
     torch.cuda.empty_cache()
     per = {k: v["total_ms"] / steps for k, v in stages.items()}
-    ix_f, at_f = indexer_flops(cfg), attn_flops(cfg)
     fp8_peak = 2.0 * peaks["bf16_sustained"]
     ix_ms = per["indexer"] + (0.0 if fused else per["topk"])
+    stage_names = ({"indexer_topk_fused": per["indexer"], "attention": per["attn"]}
+                   if fused else {"indexer": per["indexer"], "topk": per["topk"],
+                                  "attention": per["attn"]})
+    if shard is not None and stages["gather"]["launches"]:
+        stage_names["key_all_gather"] = per["gather"]
     res = {"ms_per_step": ms, "tokens_per_s": cfg.batch * cfg.n_q / (ms / 1e3),
-           "stages_ms": ({"indexer_topk_fused": per["indexer"], "attention": per["attn"]}
-                         if fused else {"indexer": per["indexer"], "topk": per["topk"],
-                                        "attention": per["attn"]}),
+           "rows_this_rank": rows,
+           "stages_ms": stage_names,
            "stage_sum_ms": sum(per.values()),
            "indexer_tflops_fp8": ix_f / (ix_ms / 1e3) / 1e12,
            "attention_tflops_bf16": at_f / (per["attn"] / 1e3) / 1e12,
@@ -432,19 +483,39 @@ def decode_leg(cfg, seed, steps, warmup, dist, peaks):
 
 # ---------------------------------------------------------------- e2e
 
-def e2e(cfg, seed, steps, dist):
+def e2e(cfg, seed, steps, dist, shard=None):
     """Same path through the public dsa_forward call with HOST buffers:
     every step copies the inputs host->device from pinned memory, runs the
-    forward and reads the result (out, lse, indices) back."""
+    forward and reads the result (out, lse, indices) back. Sharded: each
+    rank copies its rows' query inputs and its slice of the keys, the keys
+    are all-gathered on the GPUs, and each rank reads back its rows."""
     import torch
     import sparse_attention_long_fp8_b200 as dsa
+    from sparse_attention_long_fp8_b200 import inputs, shard as shard_mod
     dev_inp = dsa.make_inputs(cfg, seed=seed, device="cuda")
-    keys = ["q_fp8", "q_scale", "w", "k_fp8", "k_scale", "q_pos0", "kv_len", "q", "kv"]
-    host = {k: torch.empty(dev_inp[k].shape, dtype=dev_inp[k].dtype, pin_memory=True) for k in keys}
-    for k in keys:
-        host[k].copy_(dev_inp[k])
-    dev = {k: torch.empty_like(dev_inp[k]) for k in keys}
+    layout, kslice, full_n_kv = None, None, cfg.n_kv
+    if shard is not None:
+        rank, ranks = shard
+        rows = shard_mod.shard_rows(cfg.n_q, ranks, rank)
+        dev_inp = shard_mod.shard_inputs(dev_inp, rows)
+        cfg = inputs.custom_config(cfg.name, n_q=len(rows), name=f"{cfg.name}_shard{rank}")
+        if dist is not None:
+            kslice = shard_mod.key_slice(cfg.n_kv, ranks, rank)
+    qkeys = ["q_fp8", "q_scale", "w", "q_pos0", "kv_len", "q"] + (["row_pos"] if shard else [])
+    kkeys = ["k_fp8", "k_scale", "kv"]
+    host = {}
+    for k in qkeys + kkeys:
+        t = dev_inp[k]
+        if kslice is not None and k in kkeys:
+            t = t[:, kslice[0]:kslice[1]]
+        host[k] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        host[k].copy_(t)
+    dev = {k: torch.empty_like(dev_inp[k]) for k in qkeys + kkeys}
+    dev_local = ({k: torch.empty(host[k].shape, dtype=host[k].dtype, device="cuda") for k in kkeys}
+                 if kslice is not None else None)
     del dev_inp
+    if shard is not None:
+        layout = dsa.make_layout(row_pos=dev["row_pos"])
     shape = dsa.shape_of(cfg)
     B, T = cfg.batch, cfg.n_q
     out = torch.empty(B, T, cfg.heads, cfg.v_dim, device="cuda")
@@ -454,15 +525,21 @@ def e2e(cfg, seed, steps, dist):
     h_lse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     h_idx = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
     ws, n = dsa.alloc_workspace(shape, dsa.DSA_OP_FORWARD)
-    h2d = sum(host[k].numel() * host[k].element_size() for k in keys)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in (h_out, h_lse, h_idx))
 
     def one():
-        for k in keys:
+        for k in qkeys:
             dev[k].copy_(host[k], non_blocking=True)
+        for k in kkeys:
+            if dev_local is None:
+                dev[k].copy_(host[k], non_blocking=True)
+            else:
+                dev_local[k].copy_(host[k], non_blocking=True)
+                dev[k].copy_(shard_mod.all_gather_keys(dev_local[k], full_n_kv, dist))
         dsa.dsa_forward(shape, dev["q_fp8"], dev["q_scale"], dev["w"], dev["k_fp8"],
                         dev["k_scale"], dev["q_pos0"], dev["kv_len"], dev["q"], dev["kv"], idx,
-                        out, lse, ws, n)
+                        out, lse, ws, n, layout=layout)
         h_out.copy_(out, non_blocking=True)
         h_lse.copy_(lse, non_blocking=True)
         h_idx.copy_(idx, non_blocking=True)
@@ -481,7 +558,7 @@ def e2e(cfg, seed, steps, dist):
     torch.cuda.synchronize()
     dsa.dsa_check()
     ms = max_over_ranks(s.elapsed_time(e) / steps, dist)
-    del host, dev, out, lse, idx, h_out, h_lse, h_idx, ws
+    del host, dev, out, lse, idx, h_out, h_lse, h_idx, ws, dev_local
     torch.cuda.empty_cache()
     return ms, h2d, d2h
 
@@ -566,22 +643,29 @@ def main():
     dsa.load_library()
     torch.cuda.set_device(local)
     dist = None
-    if world > 1:
+    if world > 1 or (args.shard and "MASTER_ADDR" in os.environ):
+        # (a one-rank group under torchrun with --shard runs the all-gather too)
         import torch.distributed as tdist
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                  device_id=torch.device("cuda", local))
         dist = tdist
     peaks = measured_peaks()
     cfg = inputs.CONFIGS[args.workload]
-    seed = 1000 + rank
+    # Several GPUs split ONE prefill by query rows (strong scaling): every
+    # rank draws the same inputs and takes its share of the rows. --shard
+    # runs that path on a single rank too.
+    sharded = (world > 1 or args.shard) and not cfg.decode
+    shard = (rank, world) if sharded else None
+    seed = 1000 if sharded else 1000 + rank
 
     clocks = ClockSampler(local)
     clocks.start()
-    head, stages, fused = prefill_leg(cfg, seed, args.steps, args.warmup, dist, peaks)
+    head, stages, fused = prefill_leg(cfg, seed, args.steps, args.warmup, dist, peaks, shard)
     clock_info = clocks.stop()
     ms = head["ms_per_step"]
     tokens = cfg.batch * cfg.n_q
-    value = world * tokens / (ms / 1e3)
+    # sharded: the ranks together finish one prefill per step
+    value = (1 if sharded else world) * tokens / (ms / 1e3)
 
     per = {k: v["total_ms"] / args.steps for k, v in stages.items()}
     at_ms, ix_ms = per["attn"], per["indexer"]
@@ -612,10 +696,11 @@ def main():
     result = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": True, "scaling": "strong" if sharded else "weak",
+        "vs_baseline": None,
         "dtype": "fp8e4m3 indexer, bf16 attention, fp32 accumulate",
         "data": "synthetic (seeded; page-shaped workloads)",
-        "config": bench_config(cfg, world),
+        "config": bench_config(cfg, world, sharded),
         "stages_ms": head["stages_ms"], "stage_sum_ms": head["stage_sum_ms"],
         "indexer_tflops_fp8": head["indexer_tflops_fp8"],
         "indexer_frac_fp8": head["indexer_frac_fp8"],
@@ -627,20 +712,23 @@ def main():
 
     if not args.no_decode and args.workload == HEADLINE:
         pcfg = inputs.CONFIGS["prefill_16k"]
-        leg, _, _ = prefill_leg(pcfg, seed, args.steps, args.warmup, dist, peaks)
+        leg, _, _ = prefill_leg(pcfg, seed, args.steps, args.warmup, dist, peaks, shard)
+        leg["tokens_per_s"] = pcfg.n_q * (1 if sharded else world) / (leg["ms_per_step"] / 1e3)
         result["prefill_16k"] = leg
         result["quantiser"] = quantiser_bench(cfg, peaks)
         result["decode"] = {}
         for name in ("decode_32k", "decode_64k"):
-            # decode steps are ~0.2 ms: many of them, after a longer warm-up
-            result["decode"][name] = decode_leg(inputs.CONFIGS[name], seed,
+            # decode steps are ~0.2 ms: many of them, after a longer warm-up;
+            # under several ranks each rank decodes its own batch (weak)
+            result["decode"][name] = decode_leg(inputs.CONFIGS[name], 1000 + rank,
                                                 max(args.steps, 100), max(args.warmup, 20),
                                                 dist, peaks)
+            result["decode"][name]["scaling"] = "weak"
             torch.cuda.empty_cache()
 
     # The ranks of a node share its host RAM: every rank needs its own pinned
     # copy, and all ranks must agree before any of them enters e2e().
-    need = e2e_host_bytes(cfg)
+    need = e2e_host_bytes(cfg) // (world if sharded else 1)
     avail = host_available_bytes()
     fits = avail is None or avail >= 2 * need * world
     fits = all_ranks(fits, dist)
@@ -650,8 +738,9 @@ def main():
                                                     f"{avail / 2**30:.0f} GiB") +
                                     f" available, {world * need / 2**30:.0f} GiB pinned needed"}
     elif not args.no_e2e:
-        e_ms, h2d, d2h = e2e(cfg, seed, max(2, min(args.steps, 3)), dist)
-        result["e2e"] = {"value": world * tokens / (e_ms / 1e3), "unit": "tokens/s",
+        e_ms, h2d, d2h = e2e(cfg, seed, max(2, min(args.steps, 3)), dist, shard)
+        result["e2e"] = {"value": (1 if sharded else world) * tokens / (e_ms / 1e3),
+                         "unit": "tokens/s",
                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                          "ms_per_step": e_ms}
 
@@ -678,12 +767,13 @@ def main():
         print(json.dumps(result), flush=True)
 
 
-def bench_config(cfg, world):
+def bench_config(cfg, world, sharded=False):
     """The workload description both arms print."""
     return {"workload": cfg.name, "batch": cfg.batch, "seq_len": cfg.n_q,
             "idx_heads": cfg.idx_heads, "idx_dim": cfg.idx_dim, "topk": cfg.topk,
             "heads": cfg.heads, "qk_dim": cfg.qk_dim, "v_dim": cfg.v_dim,
-            "parallelism": f"replicas x{world}",
+            "parallelism": (f"query-sharded x{world} (one prefill; keys all-gathered)"
+                            if sharded else f"replicas x{world}"),
             "l2": "inputs larger than L2 (q is 9.7 GB per step)"}
 
 
