@@ -236,6 +236,32 @@ dsa_status set_smem(K kernel, int bytes, int dev, std::atomic<bool>* done_flags)
 
 // ------------------------------------------------------------------ indexer launch
 
+// Key tiles per CTA of the score kernel. The kernel streams key tiles from
+// HBM, so the grid is sized by its wave count: the split that minimises
+// (waves) x (tiles per CTA + a setup cost of about two tiles), with as many
+// CTAs resident per SM as shared memory and TMEM allow, and at least 4 tiles
+// per CTA to amortise the setup.
+int indexer_tiles_per_split(int n_tiles, int64_t groups, int smem_bytes, uint32_t tmem_cols) {
+  constexpr int kSmemPerSm = 233472;           // shared memory of one SM
+  const int per_sm = std::max(1, std::min(kSmemPerSm / (smem_bytes + 1024),
+                                          static_cast<int>(512 / tmem_cols)));
+  const int64_t slots = static_cast<int64_t>(per_sm) * num_sms();
+  int best_tps = n_tiles;
+  int64_t best_cost = -1;
+  for (int want = 1; want <= std::min(n_tiles, 256); ++want) {
+    const int tps = (n_tiles + want - 1) / want;
+    if (tps < 4 && tps < n_tiles) break;
+    const int splits = (n_tiles + tps - 1) / tps;
+    const int64_t waves = (groups * splits + slots - 1) / slots;
+    const int64_t cost = waves * (tps + 2);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_tps = tps;
+    }
+  }
+  return best_tps;
+}
+
 template <int HI, int DI, int QG>
 dsa_status launch_indexer_t(const dsa_shape* s, const HostLayout& lay, const uint8_t* q_fp8,
                             const float* q_scale, const float* w, const uint8_t* k_fp8,
@@ -267,11 +293,7 @@ dsa_status launch_indexer_t(const dsa_shape* s, const HostLayout& lay, const uin
   p.n_groups = (rows + QG - 1) / QG;
   const int n_tiles = (s->n_kv + T::M - 1) / T::M;
   const int64_t groups = static_cast<int64_t>(s->batch) * p.n_groups;
-  const int sms = num_sms();
-  int64_t tps = (groups * n_tiles + 4 * sms - 1) / (4 * sms);
-  tps = std::max<int64_t>(4, std::min<int64_t>(tps, 64));
-  tps = std::min<int64_t>(tps, n_tiles);
-  p.tiles_per_split = static_cast<int32_t>(tps);
+  p.tiles_per_split = indexer_tiles_per_split(n_tiles, groups, T::SMEM_BYTES, T::TMEM_COLS);
   p.write_invalid = write_invalid;
   const int n_splits = (n_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
   if (p.n_groups > 65535 || s->batch > 65535)

@@ -4,11 +4,13 @@
 //
 // One CTA per score row. Scores are mapped to order-preserving uint32 keys
 // (larger float <=> larger key; -0 is folded into +0).
-//   1. 1024 evenly spaced keys of the row are sorted (bitonic, shared
-//      memory) and a threshold tau is read off at about 1.25 k / n of the
-//      way down, so that roughly 1.25 k keys of the row are >= tau.
-//   2. One pass over the row appends every (key, index) with key >= tau to a
-//      candidate buffer in shared memory (warp-aggregated slots).
+//   1. A threshold tau from 1024 evenly spaced samples of the row: two 8-bit
+//      radix passes over the samples find the 16-bit key prefix of the
+//      sample ranked about 1.25 k / n of the way down; tau is the lowest key
+//      with that prefix, so roughly 1.25 k keys of the row are >= tau.
+//   2. One pass over the row (16-byte loads, 16 scores per thread in flight)
+//      appends every (key, index) with key >= tau to a candidate buffer in
+//      shared memory (warp-aggregated slots).
 //   3. If k <= #candidates <= capacity, an MSB-first radix select over the
 //      candidates finds the exact k-th key u*; every candidate above u* is
 //      written, then the lowest-index candidates equal to u*.
@@ -53,12 +55,14 @@ struct TopkSmem {
 // Exact k-th largest key among `n` keys given by get(i) (all threads of the
 // CTA call this). Returns u*; *need_out = number of keys equal to u* that
 // belong to the top k; *eq_out = number of keys equal to u*.
+// With passes < 4 only the top 8 * passes bits are resolved: the result is
+// that prefix (low bits zero) of the k-th largest key.
 template <class Get>
 __device__ uint32_t radix_kth(TopkSmem& sm, int n, uint32_t k, Get get, uint32_t* need_out,
-                              uint32_t* eq_out) {
+                              uint32_t* eq_out, int passes = 4) {
   const int tid = threadIdx.x;
   uint32_t prefix = 0, mask = 0, need = k, eq_count = 0;
-  for (int pass = 0; pass < 4; ++pass) {
+  for (int pass = 0; pass < passes; ++pass) {
     const int shift = 24 - 8 * pass;
     for (int i = tid; i < 256; i += kTopkThreads) sm.hist[i] = 0;
     __syncthreads();
@@ -131,51 +135,68 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
     return;
   }
 
-  // ---- 1. threshold from a sorted sample (descending)
+  // ---- 1. threshold: the 16-bit key prefix of the sample of rank `want`
   sm.samp[tid] = order_key(row[static_cast<int>((static_cast<int64_t>(tid) * n) / kTopkSamples)]);
   if (tid == 0) sm.n_cand = 0;
   __syncthreads();
-  for (int size = 2; size <= kTopkSamples; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      const int j = tid ^ stride;
-      if (j > tid) {
-        const uint32_t a = sm.samp[tid], c = sm.samp[j];
-        const bool desc = (tid & size) == 0;
-        if (desc ? (a < c) : (a > c)) {
-          sm.samp[tid] = c;
-          sm.samp[j] = a;
-        }
-      }
-      __syncthreads();
-    }
-  }
   const int64_t want =
       (static_cast<int64_t>(5) * p.k * kTopkSamples) / (4 * static_cast<int64_t>(n)) + 8;
-  const uint32_t tau = sm.samp[want < kTopkSamples - 1 ? want : kTopkSamples - 1];
+  uint32_t s_need, s_eq;
+  const uint32_t tau = radix_kth(
+      sm, kTopkSamples, static_cast<uint32_t>(want < kTopkSamples ? want : kTopkSamples),
+      [&](int i) { return sm.samp[i]; }, &s_need, &s_eq, 2);
 
-  // ---- 2. one pass: candidates >= tau (four independent loads per thread
-  // and round, so the L2 latency of the scores overlaps)
-  for (int c0 = 0; c0 < n; c0 += 4 * kTopkThreads) {
-    uint32_t u[4];
+  // ---- 2. one pass: candidates >= tau. Sixteen scores per thread and round
+  // are loaded before any is appended, as four 16-byte loads when the row is
+  // 16-byte aligned, so that the L2 / HBM latency of the row overlaps.
+  auto append = [&](uint32_t u, int i) {
+    const bool take = i < n && u >= tau;
+    const uint32_t bal = __ballot_sync(0xffffffffu, take);
+    if (bal) {
+      uint32_t base = 0;
+      if (lane == 0) base = atomicAdd(&sm.n_cand, static_cast<uint32_t>(__popc(bal)));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      const uint32_t slot = base + __popc(bal & ((1u << lane) - 1u));
+      if (take && slot < static_cast<uint32_t>(kTopkCap)) {
+        sm.cand_u[slot] = u;
+        sm.cand_i[slot] = i;
+      }
+    }
+  };
+  int scalar_from = 0;   // scores [scalar_from, n) take the scalar loop
+  if ((reinterpret_cast<uintptr_t>(row) & 15u) == 0) {
+    // whole float4s inside [0, n) only; the tail (< 4 scores) below
+    const float4* row4 = reinterpret_cast<const float4*>(row);
+    const int n4 = n >> 2;
+    scalar_from = n4 * 4;
+    for (int c0 = 0; c0 < n4; c0 += 4 * kTopkThreads) {
+      float4 v[4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
+      for (int m = 0; m < 4; ++m) {
+        const int c = c0 + tid + m * kTopkThreads;
+        v[m] = c < n4 ? row4[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        // past the last whole float4: an index >= n, so nothing is appended
+        const int c = c0 + tid + m * kTopkThreads;
+        const int i = c < n4 ? c * 4 : n;
+        append(order_key(v[m].x), i);
+        append(order_key(v[m].y), i + 1);
+        append(order_key(v[m].z), i + 2);
+        append(order_key(v[m].w), i + 3);
+      }
+    }
+  }
+  for (int c0 = scalar_from; c0 < n; c0 += 16 * kTopkThreads) {
+    uint32_t u[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
       const int i = c0 + tid + m * kTopkThreads;
       u[m] = i < n ? order_key(row[i]) : 0u;
     }
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const int i = c0 + tid + m * kTopkThreads;
-      const bool take = i < n && u[m] >= tau;
-      const uint32_t bal = __ballot_sync(0xffffffffu, take);
-      uint32_t base = 0;
-      if (lane == 0 && bal) base = atomicAdd(&sm.n_cand, static_cast<uint32_t>(__popc(bal)));
-      base = __shfl_sync(0xffffffffu, base, 0);
-      const uint32_t slot = base + __popc(bal & ((1u << lane) - 1u));
-      if (take && slot < static_cast<uint32_t>(kTopkCap)) {
-        sm.cand_u[slot] = u[m];
-        sm.cand_i[slot] = i;
-      }
-    }
+    for (int m = 0; m < 16; ++m) append(u[m], c0 + tid + m * kTopkThreads);
   }
   __syncthreads();
   const uint32_t n_cand = sm.n_cand;
