@@ -317,14 +317,20 @@ void oracle_indexer_kl(int n_rows, int S, int HI, int DI, const uint8_t* q8, con
       }
       for (int s = 0; s < n_vis; ++s) p[s] += z[s] / l / static_cast<double>(H);
     }
-    // indexer scores I (direct form) and x kept for the gradient
+    // indexer scores I and x kept for the gradient. x = q^ . k^ is formed
+    // as (sum_d code_q code_k) * q_scale * k_scale: the code products are
+    // exact in fp64 and so is their sum (at most 128 terms spanning 36 bits),
+    // so the sign of x, which decides the ReLU and its mask, is exact.
     std::vector<double> x(static_cast<size_t>(n_vis) * HI), I(n_vis);
     for (int s = 0; s < n_vis; ++s) {
       double score = 0.0;
       for (int j = 0; j < HI; ++j) {
-        double dot = 0.0;
+        double code_dot = 0.0;
         for (int d = 0; d < DI; ++d)
-          dot += qhat[static_cast<size_t>(j) * DI + d] * khat[static_cast<size_t>(s) * DI + d];
+          code_dot += e4m3_value(q8[(static_cast<size_t>(r) * HI + j) * DI + d]) *
+                      e4m3_value(k8[static_cast<size_t>(s) * DI + d]);
+        const double dot = code_dot * static_cast<double>(qs[static_cast<size_t>(r) * HI + j]) *
+                           static_cast<double>(ks[s]);
         x[static_cast<size_t>(s) * HI + j] = dot;
         score += static_cast<double>(w[static_cast<size_t>(r) * HI + j]) * (dot > 0.0 ? dot : 0.0);
       }
