@@ -71,7 +71,8 @@ typedef enum {
   DSA_OP_INDEXER = 0,
   DSA_OP_TOPK = 1,
   DSA_OP_SPARSE_ATTN = 2,
-  DSA_OP_FORWARD = 3
+  DSA_OP_FORWARD = 3,
+  DSA_OP_INDEXER_KL = 4
 } dsa_op;
 
 typedef struct {
@@ -294,6 +295,38 @@ dsa_status dsa_forward_ex(const dsa_shape* shape, const dsa_layout* layout,
                           const uint16_t* q, const uint16_t* kv,
                           int32_t* indices_out, void* out, int32_t out_dtype,
                           float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Indexer warm-up loss and its gradient (page "DeepseekV3.2 拆解", section
+ * "预训练策略 / 密集预热阶段": with the main model frozen, the indexer is
+ * trained to follow the dense attention distribution,
+ *     L^I = sum_t KL(p_{t,:} || Softmax(I_{t,:}))).
+ *   p_{t,:}   the main attention's dense causal softmax of query row t over
+ *             its visible keys (softmax_scale * q . kv over all qk_dim
+ *             dims), averaged over the H heads;
+ *   I_{t,:}   the indexer scores of dsa_indexer_scores over the same keys.
+ *   Inputs:   the indexer inputs of dsa_indexer_scores (all n_q rows) and the
+ *             attention inputs q [B, n_q, H, D_qk], kv [B, n_kv, D_qk] bf16.
+ *   Outputs (fp32, written in full):
+ *     loss [B, n_q]          KL of each row (sum them for L^I);
+ *     dw   [B, n_q, H^I]     dL/dw;
+ *     dq   [B, n_q, H^I, d^I] dL/dq^ with q^ = code * q_scale (the FP8
+ *                            encoding passes the gradient through);
+ *     dk   [B, n_kv, d^I]    dL/dk^ with k^ = code * k_scale (zero for keys
+ *                            no row sees).
+ *   p on the tensor cores (bf16, fp32 accumulate); the loss rows and the
+ *   gradient sums in fp32. The ReLU mask [q^ . k^ > 0] is the sign of the
+ *   tensor-core dot product (exact products, fp32 sum).
+ *   Workspace: dsa_workspace_size(shape, DSA_OP_INDEXER_KL) bytes (16 per
+ *   (row, key) of a row chunk), 256-byte aligned. Contiguous caches only.
+ */
+dsa_status dsa_indexer_kl(const dsa_shape* shape, const uint8_t* q_fp8,
+                          const float* q_scale, const float* w,
+                          const uint8_t* k_fp8, const float* k_scale,
+                          const int32_t* q_pos0, const int32_t* kv_len,
+                          const uint16_t* q, const uint16_t* kv,
+                          float* loss, float* dw, float* dq, float* dk,
+                          void* ws, size_t ws_bytes, void* stream);
 
 /* Rows per indexer/top-k step that dsa_forward uses for this shape. With
  * the fused plan it is n_q (one dsa_indexer_topk launch over all rows, no

@@ -34,6 +34,7 @@ DSA_OP_INDEXER = 0
 DSA_OP_TOPK = 1
 DSA_OP_SPARSE_ATTN = 2
 DSA_OP_FORWARD = 3
+DSA_OP_INDEXER_KL = 4
 
 
 class DsaError(RuntimeError):
@@ -97,6 +98,7 @@ def load_library(path: str | None = None):
     lib.dsa_sparse_attn_noalloc.argtypes = [SP, P, P, P, P, I32, P, P]
     lib.dsa_forward.argtypes = [SP, P, P, P, P, P, P, P, P, P, P, P, I32, P, P, SZ, P]
     lib.dsa_workspace_size.argtypes = [SP, I32, ctypes.POINTER(SZ)]
+    lib.dsa_indexer_kl.argtypes = [SP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
     lib.dsa_check.argtypes = [P]
     lib.dsa_quantize_e4m3.argtypes = [ctypes.c_int64, I32, P, P, P, P]
     lib.dsa_quantize_e4m3.restype = ctypes.c_int
@@ -118,7 +120,8 @@ def load_library(path: str | None = None):
     for fn in ("dsa_indexer_scores", "dsa_indexer_topk", "dsa_topk", "dsa_sparse_attn", "dsa_forward",
                "dsa_workspace_size", "dsa_check", "dsa_forward_chunk_rows",
                "dsa_sparse_attn_noalloc", "dsa_forward_plan", "dsa_indexer_scores_ex",
-               "dsa_indexer_topk_ex", "dsa_topk_ex", "dsa_sparse_attn_ex", "dsa_forward_ex"):
+               "dsa_indexer_topk_ex", "dsa_topk_ex", "dsa_sparse_attn_ex", "dsa_forward_ex",
+               "dsa_indexer_kl"):
         getattr(lib, fn).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -283,6 +286,36 @@ def dsa_forward(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, q, kv,
         _ptr(indices_out, d["i32"], "indices_out"),
         _ptr(out, (torch.float32, torch.bfloat16), "out"), out_dtype,
         _ptr(lse, d["f32"], "lse"), _ptr(ws, None, "ws"), int(ws_bytes), _stream(stream)))
+
+
+def dsa_indexer_kl(shape, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, q, kv,
+                   loss, dw, dq, dk, ws=None, ws_bytes=0, stream=None):
+    d = _dt()
+    _raise(load_library().dsa_indexer_kl(
+        ctypes.byref(shape), _ptr(q_fp8, d["u8"], "q_fp8"), _ptr(q_scale, d["f32"], "q_scale"),
+        _ptr(w, d["f32"], "w"), _ptr(k_fp8, d["u8"], "k_fp8"), _ptr(k_scale, d["f32"], "k_scale"),
+        _ptr(q_pos0, d["i32"], "q_pos0"), _ptr(kv_len, d["i32"], "kv_len"),
+        _ptr(q, d["bf16"], "q"), _ptr(kv, d["bf16"], "kv"), _ptr(loss, d["f32"], "loss"),
+        _ptr(dw, d["f32"], "dw"), _ptr(dq, d["f32"], "dq"), _ptr(dk, d["f32"], "dk"),
+        _ptr(ws, None, "ws"), int(ws_bytes), _stream(stream)))
+
+
+def indexer_kl(inp: dict, cfg: DsaConfig, stream=None):
+    """The warm-up loss and gradient on CUDA tensors from ``make_inputs``;
+    returns dict(loss, dw, dq, dk). Buffers are allocated with torch."""
+    import torch
+    shape = shape_of(cfg)
+    dev = inp["q"].device
+    B, T, S = cfg.batch, cfg.n_q, cfg.n_kv
+    loss = torch.empty(B, T, device=dev)
+    dw = torch.empty(B, T, cfg.idx_heads, device=dev)
+    dq = torch.empty(B, T, cfg.idx_heads, cfg.idx_dim, device=dev)
+    dk = torch.empty(B, S, cfg.idx_dim, device=dev)
+    ws, n = alloc_workspace(shape, DSA_OP_INDEXER_KL, dev)
+    dsa_indexer_kl(shape, inp["q_fp8"], inp["q_scale"], inp["w"], inp["k_fp8"], inp["k_scale"],
+                   inp["q_pos0"], inp["kv_len"], inp["q"], inp["kv"], loss, dw, dq, dk, ws, n,
+                   stream)
+    return {"loss": loss, "dw": dw, "dq": dq, "dk": dk}
 
 
 def dsa_check(stream=None):

@@ -22,6 +22,7 @@
 #include "topk.cuh"
 #include "selftest.cuh"
 #include "quantize.cuh"
+#include "indexer_kl.cuh"
 
 namespace {
 
@@ -267,7 +268,7 @@ dsa_status launch_indexer_t(const dsa_shape* s, const HostLayout& lay, const uin
                             const float* q_scale, const float* w, const uint8_t* k_fp8,
                             const float* k_scale, const int32_t* q_pos0, const int32_t* kv_len,
                             int32_t row_begin, int32_t rows, float* scores, int write_invalid,
-                            cudaStream_t stream, int dev) {
+                            cudaStream_t stream, int dev, uint64_t* signs = nullptr) {
   using T = dsa::IndexerTile<HI, DI, QG>;
   static std::atomic<bool> attr_done[kMaxDevices];
   if (dsa_status st = set_smem(dsa::indexer_scores_kernel<HI, DI, QG>, T::SMEM_BYTES, dev, attr_done))
@@ -285,6 +286,7 @@ dsa_status launch_indexer_t(const dsa_shape* s, const HostLayout& lay, const uin
   p.km = lay.km;
   p.kv_len = kv_len;
   p.scores = scores;
+  p.signs = signs;
   p.B = s->batch;
   p.n_q = s->n_q;
   p.n_kv = s->n_kv;
@@ -308,20 +310,20 @@ dsa_status launch_indexer(const dsa_shape* s, const HostLayout& lay, const uint8
                           const float* q_scale, const float* w, const uint8_t* k_fp8,
                           const float* k_scale, const int32_t* q_pos0, const int32_t* kv_len,
                           int32_t row_begin, int32_t rows, float* scores, int write_invalid,
-                          cudaStream_t stream, int dev) {
+                          cudaStream_t stream, int dev, uint64_t* signs = nullptr) {
   if (s->idx_heads == 64) {
     if (rows == 1)
       return launch_indexer_t<64, 128, 1>(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0,
                                           kv_len, row_begin, rows, scores, write_invalid, stream,
-                                          dev);
+                                          dev, signs);
     return launch_indexer_t<64, 128, 4>(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
-                                        row_begin, rows, scores, write_invalid, stream, dev);
+                                        row_begin, rows, scores, write_invalid, stream, dev, signs);
   }
   if (rows <= 4)
     return launch_indexer_t<4, 32, 4>(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
-                                      row_begin, rows, scores, write_invalid, stream, dev);
+                                      row_begin, rows, scores, write_invalid, stream, dev, signs);
   return launch_indexer_t<4, 32, 64>(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
-                                     row_begin, rows, scores, write_invalid, stream, dev);
+                                     row_begin, rows, scores, write_invalid, stream, dev, signs);
 }
 
 // Scores and selection in one kernel: H^I = 64, d^I = 128, k <= 2048.
@@ -565,6 +567,75 @@ FwdPlan plan_forward(const dsa_shape* s) {
   return f;
 }
 
+// ------------------------------------------------------------------ warm-up loss plan
+
+// Rows per chunk of dsa_indexer_kl: per (row, key) it stores p (then g), the
+// score I and the sign mask, 16 bytes; a chunk of every sequence's rows
+// takes at most ~512 MB of workspace.
+struct KlPlan {
+  int chunk_rows;
+  size_t pbar_bytes, scores_bytes, signs_bytes, total;
+};
+
+KlPlan plan_kl(const dsa_shape* s) {
+  KlPlan k{};
+  const size_t per_row = static_cast<size_t>(s->batch) * s->n_kv;
+  const size_t budget = 512ull << 20;
+  int64_t chunk = static_cast<int64_t>(budget / (16 * per_row));
+  chunk = std::max<int64_t>(1, std::min<int64_t>(chunk, s->n_q));
+  k.chunk_rows = static_cast<int>(chunk);
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  k.pbar_bytes = up(per_row * chunk * 4);
+  k.scores_bytes = up(per_row * chunk * 4);
+  k.signs_bytes = up(per_row * chunk * 8);
+  k.total = k.pbar_bytes + k.scores_bytes + k.signs_bytes;
+  return k;
+}
+
+dsa_status check_kl_shape(const dsa_shape* s) {
+  if (dsa_status st = check_indexer_shape(s)) return st;
+  if (dsa_status st = check_attn_shape(s)) return st;
+  return DSA_OK;
+}
+
+template <int DQK>
+dsa_status launch_kl_probs(const dsa_shape* s, const uint16_t* q, const uint16_t* kv,
+                           const int32_t* q_pos0, const int32_t* kv_len, int32_t row_begin,
+                           int32_t rows, float* pbar, cudaStream_t stream, int dev) {
+  using T = dsa::KlProbTile<DQK>;
+  static std::atomic<bool> attr_done[kMaxDevices];
+  if (dsa_status st = set_smem(dsa::kl_probs_kernel<DQK>, T::SMEM_BYTES, dev, attr_done)) return st;
+  dsa::KlProbParams p{};
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.kv = reinterpret_cast<const __nv_bfloat16*>(kv);
+  p.q_pos0 = q_pos0;
+  p.kv_len = kv_len;
+  p.pbar = pbar;
+  p.B = s->batch;
+  p.n_q = s->n_q;
+  p.n_kv = s->n_kv;
+  p.H = s->heads;
+  p.row_begin = row_begin;
+  p.rows = rows;
+  p.scale_log2 = s->softmax_scale * 1.4426950408889634f;
+  dim3 grid(rows, s->batch);
+  dsa::kl_probs_kernel<DQK><<<grid, T::THREADS, T::SMEM_BYTES, stream>>>(p);
+  DSA_CUDA_TRY(cudaGetLastError(), "warm-up loss probabilities launch");
+  return DSA_OK;
+}
+
+template <int HI, int DI>
+dsa_status launch_kl_grads(const dsa::KlGradParams& p, int32_t rows, int32_t batch, int32_t n_kv,
+                           cudaStream_t stream) {
+  using Map = dsa::KlGradUMap<HI, DI>;
+  dsa::kl_grad_u_kernel<HI, DI><<<dim3(rows, batch), Map::THREADS, 0, stream>>>(p);
+  DSA_CUDA_TRY(cudaGetLastError(), "warm-up loss gradient (q, w) launch");
+  dsa::kl_grad_k_kernel<HI, DI>
+      <<<dim3((n_kv + 31) / 32, batch), dsa::kKlGradThreads, 0, stream>>>(p);
+  DSA_CUDA_TRY(cudaGetLastError(), "warm-up loss gradient (k) launch");
+  return DSA_OK;
+}
+
 dsa_status check_ptrs(std::initializer_list<const void*> ptrs, const char* what) {
   for (const void* p : ptrs)
     if (!p) return fail(DSA_ERR_INVALID_ARG, "%s: required pointer is NULL", what);
@@ -675,6 +746,11 @@ dsa_status dsa_workspace_size(const dsa_shape* s, int32_t op, size_t* bytes) {
       if (dsa_status st = check_indexer_shape(s)) return st;
       if (dsa_status st = check_attn_shape(s)) return st;
       *bytes = plan_forward(s).total;
+      return DSA_OK;
+    }
+    case DSA_OP_INDEXER_KL: {
+      if (dsa_status st = check_kl_shape(s)) return st;
+      *bytes = plan_kl(s).total;
       return DSA_OK;
     }
     default:
@@ -907,6 +983,85 @@ dsa_status dsa_forward(const dsa_shape* s, const uint8_t* q_fp8, const float* q_
                        float* lse, void* ws, size_t ws_bytes, void* stream) {
   return dsa_forward_ex(s, nullptr, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len, q, kv,
                         indices_out, out, out_dtype, lse, ws, ws_bytes, stream);
+}
+
+dsa_status dsa_indexer_kl(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,
+                          const float* w, const uint8_t* k_fp8, const float* k_scale,
+                          const int32_t* q_pos0, const int32_t* kv_len, const uint16_t* q,
+                          const uint16_t* kv, float* loss, float* dw, float* dq, float* dk,
+                          void* ws, size_t ws_bytes, void* stream) {
+  if (dsa_status st = check_kl_shape(s)) return st;
+  if (dsa_status st = check_ptrs({q_fp8, q_scale, w, k_fp8, k_scale, q, kv, loss, dw, dq, dk},
+                                 "dsa_indexer_kl"))
+    return st;
+  if (!aligned(q_fp8, 16) || !aligned(k_fp8, 16) || !aligned(q, 16) || !aligned(kv, 16))
+    return fail(DSA_ERR_INVALID_ARG, "q_fp8, k_fp8, q and kv must be 16-byte aligned");
+  const KlPlan plan = plan_kl(s);
+  if (!ws || ws_bytes < plan.total)
+    return fail(DSA_ERR_WORKSPACE, "dsa_indexer_kl needs %zu workspace bytes, got %zu", plan.total,
+                ws ? ws_bytes : size_t(0));
+  if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  HostLayout lay;
+  if (dsa_status st = resolve_layout(s, nullptr, &lay)) return st;
+  int dev;
+  if (dsa_status st = current_device(&dev)) return st;
+  cudaStream_t st_ = static_cast<cudaStream_t>(stream);
+  float* pbar = static_cast<float*>(ws);
+  float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.pbar_bytes);
+  uint64_t* signs =
+      reinterpret_cast<uint64_t*>(static_cast<char*>(ws) + plan.pbar_bytes + plan.scores_bytes);
+  // dk is a sum over every row chunk
+  DSA_CUDA_TRY(cudaMemsetAsync(dk, 0,
+                               static_cast<size_t>(s->batch) * s->n_kv * s->idx_dim * sizeof(float),
+                               st_),
+               "clear dk");
+  for (int r0 = 0; r0 < s->n_q; r0 += plan.chunk_rows) {
+    const int rows = std::min(plan.chunk_rows, s->n_q - r0);
+    if (s->qk_dim == 576) {
+      if (dsa_status e = launch_kl_probs<576>(s, q, kv, q_pos0, kv_len, r0, rows, pbar, st_, dev))
+        return e;
+    } else {
+      if (dsa_status e = launch_kl_probs<64>(s, q, kv, q_pos0, kv_len, r0, rows, pbar, st_, dev))
+        return e;
+    }
+    if (dsa_status e = launch_indexer(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
+                                      r0, rows, scores, 1, st_, dev, signs))
+      return e;
+    dsa::KlRowParams rp{};
+    rp.scores = scores;
+    rp.pbar = pbar;
+    rp.loss = loss;
+    rp.q_pos0 = q_pos0;
+    rp.kv_len = kv_len;
+    rp.n_q = s->n_q;
+    rp.n_kv = s->n_kv;
+    rp.row_begin = r0;
+    rp.rows = rows;
+    dsa::kl_rows_kernel<<<dim3(rows, s->batch), dsa::kKlRowThreads, 0, st_>>>(rp);
+    DSA_CUDA_TRY(cudaGetLastError(), "warm-up loss rows launch");
+    dsa::KlGradParams gp{};
+    gp.q_fp8 = q_fp8;
+    gp.q_scale = q_scale;
+    gp.w = w;
+    gp.k_fp8 = k_fp8;
+    gp.k_scale = k_scale;
+    gp.g = pbar;
+    gp.signs = signs;
+    gp.q_pos0 = q_pos0;
+    gp.kv_len = kv_len;
+    gp.dw = dw;
+    gp.dq = dq;
+    gp.dk = dk;
+    gp.n_q = s->n_q;
+    gp.n_kv = s->n_kv;
+    gp.row_begin = r0;
+    gp.rows = rows;
+    dsa_status e = s->idx_heads == 64
+                       ? launch_kl_grads<64, 128>(gp, rows, s->batch, s->n_kv, st_)
+                       : launch_kl_grads<4, 32>(gp, rows, s->batch, s->n_kv, st_);
+    if (e) return e;
+  }
+  return DSA_OK;
 }
 
 dsa_status dsa_check(void* stream) {

@@ -31,6 +31,7 @@ struct IndexerParams {
   KeyMap km;              // pool row of each key
   const int32_t* kv_len;  // [B] or null
   float* scores;          // [B, rows, n_kv]
+  uint64_t* signs;        // [B, rows, n_kv] bit j: x[t, j, s] > 0, or null
   int32_t B, n_q, n_kv;
   int32_t row_begin, rows;     // scored rows [row_begin, row_begin + rows)
   int32_t n_groups;            // ceil(rows / QG)
@@ -226,6 +227,7 @@ __global__ void __launch_bounds__(IndexerTile<HI, DI, QG>::THREADS, 1)
         const int ql = qhalf * T::QPW + q;
         const uint32_t col = tmem_base + lane_addr + buf * T::N + ql * HI;
         float acc = 0.f;
+        uint64_t sbits = 0;   // sign of each head's dot product (training path)
         if constexpr (HI >= 32) {
 #pragma unroll
           for (int h0 = 0; h0 < HI; h0 += 32) {
@@ -235,6 +237,12 @@ __global__ void __launch_bounds__(IndexerTile<HI, DI, QG>::THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               acc = fmaf(cf[q][h0 + j], fmaxf(__uint_as_float(x[j]), 0.f), acc);
+            if (p.signs) {
+              uint32_t m = 0;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) m |= (__uint_as_float(x[j]) > 0.f ? 1u : 0u) << j;
+              sbits |= static_cast<uint64_t>(m) << h0;
+            }
           }
         } else {
           uint32_t x[4];
@@ -242,12 +250,18 @@ __global__ void __launch_bounds__(IndexerTile<HI, DI, QG>::THREADS, 1)
           tmem_ld4(col, x);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 4; ++j) acc = fmaf(cf[q][j], fmaxf(__uint_as_float(x[j]), 0.f), acc);
+          for (int j = 0; j < 4; ++j) {
+            acc = fmaf(cf[q][j], fmaxf(__uint_as_float(x[j]), 0.f), acc);
+            sbits |= static_cast<uint64_t>(__uint_as_float(x[j]) > 0.f ? 1u : 0u) << j;
+          }
         }
         const int r = r0 + ql;
         if (r <= r_last && s < p.n_kv) {
           const bool vis = s <= rpos[q] && s < kvl;
           out_base[static_cast<size_t>(ql) * row_stride + s] = vis ? acc * ks : -INFINITY;
+          if (p.signs)
+            p.signs[(static_cast<size_t>(b) * p.rows + (r0 - p.row_begin) + ql) * row_stride + s] =
+                sbits;
         }
       }
       tc_fence_before();

@@ -117,7 +117,7 @@ __device__ uint32_t radix_kth(TopkSmem& sm, int n, uint32_t k, Get get, uint32_t
   return prefix;
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 2) topk_kernel(TopkParams p) {
+__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
   extern __shared__ __align__(16) uint8_t tk_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_raw);
 
