@@ -459,6 +459,54 @@ def prefill_leg(cfg, seed, steps, warmup, dist, peaks, shard=None):
     return res, stages, fused
 
 
+def warmup_loss_flops(cfg):
+    """Algorithmic flops of one indexer warm-up loss step (dsa_indexer_kl)
+    over a causal prefill: the dense attention logits that give p
+    (2 H D_qk per visible pair), the indexer scores (2 H^I d^I per pair) and
+    the two gradient contractions U and dk (2 H^I d^I per pair each)."""
+    pairs = visible_pairs(cfg)
+    return {"probs_bf16": 2.0 * cfg.heads * cfg.qk_dim * pairs,
+            "scores_fp8": 2.0 * cfg.idx_heads * cfg.idx_dim * pairs,
+            "grads_fp32": 4.0 * cfg.idx_heads * cfg.idx_dim * pairs}
+
+
+def warmup_loss_leg(cfg, seed, steps, warmup):
+    """dsa_indexer_kl (loss + dL/dw, dL/dq^, dL/dk^) over one prefill."""
+    import torch
+    import sparse_attention_long_fp8_b200 as dsa
+    g = dsa.make_inputs(cfg, seed=seed, device="cuda")
+    shape = dsa.shape_of(cfg)
+    B, T, S = cfg.batch, cfg.n_q, cfg.n_kv
+    loss = torch.empty(B, T, device="cuda")
+    dw = torch.empty(B, T, cfg.idx_heads, device="cuda")
+    dq = torch.empty(B, T, cfg.idx_heads, cfg.idx_dim, device="cuda")
+    dk = torch.empty(B, S, cfg.idx_dim, device="cuda")
+    ws, n = dsa.alloc_workspace(shape, dsa.DSA_OP_INDEXER_KL)
+
+    def run():
+        dsa.dsa_indexer_kl(shape, g["q_fp8"], g["q_scale"], g["w"], g["k_fp8"], g["k_scale"],
+                           g["q_pos0"], g["kv_len"], g["q"], g["kv"], loss, dw, dq, dk, ws, n)
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    dsa.dsa_check()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        run()
+    e.record()
+    torch.cuda.synchronize()
+    dsa.dsa_check()
+    ms = s.elapsed_time(e) / steps
+    fl = warmup_loss_flops(cfg)
+    del g, loss, dw, dq, dk, ws
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "tokens_per_s": B * T / (ms / 1e3),
+            "algorithmic_tflop": {k: v / 1e12 for k, v in fl.items()},
+            "what": "loss and gradient w.r.t. w, q^, k^ of sum_t KL(p_t || Softmax(I_t))"}
+
+
 def decode_leg(cfg, seed, steps, warmup, dist, peaks):
     """Batch decode: dsa_forward captured in a CUDA graph (a step is ~0.2 ms
     of a few launches), bytes per step as decode_bytes counts them."""
@@ -716,6 +764,8 @@ def main():
         leg["tokens_per_s"] = pcfg.n_q * (1 if sharded else world) / (leg["ms_per_step"] / 1e3)
         result["prefill_16k"] = leg
         result["quantiser"] = quantiser_bench(cfg, peaks)
+        result["warmup_loss_4k"] = warmup_loss_leg(inputs.CONFIGS["prefill_4k"], seed,
+                                                   max(3, args.steps // 4), args.warmup)
         result["decode"] = {}
         for name in ("decode_32k", "decode_64k"):
             # decode steps are ~0.2 ms: many of them, after a longer warm-up;

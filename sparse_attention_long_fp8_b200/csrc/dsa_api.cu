@@ -573,8 +573,8 @@ FwdPlan plan_forward(const dsa_shape* s) {
 // score I and the sign mask, 16 bytes; a chunk of every sequence's rows
 // takes at most ~512 MB of workspace.
 struct KlPlan {
-  int chunk_rows;
-  size_t pbar_bytes, scores_bytes, signs_bytes, total;
+  int chunk_rows, k_split;
+  size_t pbar_bytes, scores_bytes, signs_bytes, part_bytes, total;
 };
 
 KlPlan plan_kl(const dsa_shape* s) {
@@ -588,7 +588,13 @@ KlPlan plan_kl(const dsa_shape* s) {
   k.pbar_bytes = up(per_row * chunk * 4);
   k.scores_bytes = up(per_row * chunk * 4);
   k.signs_bytes = up(per_row * chunk * 8);
-  k.total = k.pbar_bytes + k.scores_bytes + k.signs_bytes;
+  // dk partials: the chunk's rows split so that key tiles x splits fill the
+  // SMs about twice
+  const int64_t tiles = static_cast<int64_t>(s->batch) * ((s->n_kv + 63) / 64);
+  k.k_split = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>({16, chunk, (2 * num_sms() + tiles - 1) / tiles})));
+  k.part_bytes = up(static_cast<size_t>(k.k_split) * per_row * s->idx_dim * 4);
+  k.total = k.pbar_bytes + k.scores_bytes + k.signs_bytes + k.part_bytes;
   return k;
 }
 
@@ -626,13 +632,22 @@ dsa_status launch_kl_probs(const dsa_shape* s, const uint16_t* q, const uint16_t
 
 template <int HI, int DI>
 dsa_status launch_kl_grads(const dsa::KlGradParams& p, int32_t rows, int32_t batch, int32_t n_kv,
-                           cudaStream_t stream) {
+                           float* part, int32_t k_split, cudaStream_t stream, int dev) {
   using Map = dsa::KlGradUMap<HI, DI>;
+  using KMap = dsa::KlGradKMap<HI, DI>;
+  static std::atomic<bool> attr_done[kMaxDevices];
+  if (dsa_status st = set_smem(dsa::kl_grad_k_kernel<HI, DI>, KMap::SMEM_BYTES, dev, attr_done))
+    return st;
   dsa::kl_grad_u_kernel<HI, DI><<<dim3(rows, batch), Map::THREADS, 0, stream>>>(p);
   DSA_CUDA_TRY(cudaGetLastError(), "warm-up loss gradient (q, w) launch");
-  dsa::kl_grad_k_kernel<HI, DI>
-      <<<dim3((n_kv + 31) / 32, batch), dsa::kKlGradThreads, 0, stream>>>(p);
+  dsa::kl_grad_k_kernel<HI, DI><<<dim3((n_kv + KMap::KT - 1) / KMap::KT, k_split, batch),
+                                   dsa::kKlGradThreads, KMap::SMEM_BYTES, stream>>>(p, part,
+                                                                                    k_split);
   DSA_CUDA_TRY(cudaGetLastError(), "warm-up loss gradient (k) launch");
+  const int64_t n = static_cast<int64_t>(batch) * n_kv * DI;
+  const int blocks = static_cast<int>(std::min<int64_t>((n + 255) / 256, 4 * num_sms()));
+  dsa::kl_grad_k_reduce_kernel<<<blocks, 256, 0, stream>>>(part, p.dk, n, k_split);
+  DSA_CUDA_TRY(cudaGetLastError(), "warm-up loss gradient (k) reduce launch");
   return DSA_OK;
 }
 
@@ -1010,6 +1025,8 @@ dsa_status dsa_indexer_kl(const dsa_shape* s, const uint8_t* q_fp8, const float*
   float* scores = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.pbar_bytes);
   uint64_t* signs =
       reinterpret_cast<uint64_t*>(static_cast<char*>(ws) + plan.pbar_bytes + plan.scores_bytes);
+  float* part = reinterpret_cast<float*>(static_cast<char*>(ws) + plan.pbar_bytes +
+                                         plan.scores_bytes + plan.signs_bytes);
   // dk is a sum over every row chunk
   DSA_CUDA_TRY(cudaMemsetAsync(dk, 0,
                                static_cast<size_t>(s->batch) * s->n_kv * s->idx_dim * sizeof(float),
@@ -1056,9 +1073,10 @@ dsa_status dsa_indexer_kl(const dsa_shape* s, const uint8_t* q_fp8, const float*
     gp.n_kv = s->n_kv;
     gp.row_begin = r0;
     gp.rows = rows;
+    const int ksplit = std::min(plan.k_split, rows);
     dsa_status e = s->idx_heads == 64
-                       ? launch_kl_grads<64, 128>(gp, rows, s->batch, s->n_kv, st_)
-                       : launch_kl_grads<4, 32>(gp, rows, s->batch, s->n_kv, st_);
+                       ? launch_kl_grads<64, 128>(gp, rows, s->batch, s->n_kv, part, ksplit, st_, dev)
+                       : launch_kl_grads<4, 32>(gp, rows, s->batch, s->n_kv, part, ksplit, st_, dev);
     if (e) return e;
   }
   return DSA_OK;

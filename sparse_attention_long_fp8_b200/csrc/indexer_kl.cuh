@@ -442,29 +442,47 @@ __global__ void __launch_bounds__(kKlGradThreads) kl_grad_u_kernel(KlGradParams 
   }
 }
 
-// dk^[s] += sum over the chunk's rows t (s visible to t) and heads j of
-// g[t,s] w[t,j] [x > 0] q^[t,j]. One CTA per tile of KT keys; thread
-// (key k, dim group) keeps DI * KT / 256 outputs.
+// dk^[s] partial over a split of the chunk's rows: sum over rows t (s visible
+// to t) and heads j of g[t,s] w[t,j] [x > 0] q^[t,j]. Grid (key tiles of KT,
+// row splits, batch); thread (key group, dim group) keeps KPT keys x DPT
+// dims. Partials go to part[split] and kl_grad_k_reduce_kernel adds them to
+// dk in split order, so the sum is the same on every call.
 template <int HI, int DI>
-__global__ void __launch_bounds__(kKlGradThreads) kl_grad_k_kernel(KlGradParams p) {
-  constexpr int KT = 32;                            // keys per CTA
-  constexpr int NDG = kKlGradThreads / KT;          // dim groups per key
-  constexpr int DG = DI / NDG;
-  static_assert(NDG * DG == DI && DG >= 1, "thread map");
-  __shared__ float qv[HI][DI];                      // q^ of the current row
-  __shared__ float a_s[KT][HI];                     // g w [x > 0] per (key, head)
-  __shared__ float g_s[KT];                         // g[t, s] of the tile's keys
-  __shared__ unsigned long long m_s[KT];            // their sign masks
-  const int tile = blockIdx.x, b = blockIdx.y;
+struct KlGradKMap {
+  static constexpr int KT = 64;                              // keys per CTA
+  static constexpr int DPT = 8;                              // dims per thread
+  static constexpr int NDG = DI / DPT;                       // dim groups
+  static constexpr int NKG = kKlGradThreads / NDG;           // key groups
+  static constexpr int KPT = KT / NKG;                       // keys per thread
+  static_assert(NDG * DPT == DI && NKG * KPT == KT && KPT >= 1, "thread map");
+  // dynamic shared memory: q^ [HI][DI], a [HI][KT], g [KT], masks [KT]
+  static constexpr int SMEM_BYTES = (HI * DI + HI * KT + KT) * 4 + KT * 8;
+};
+
+template <int HI, int DI>
+__global__ void __launch_bounds__(kKlGradThreads) kl_grad_k_kernel(KlGradParams p, float* part,
+                                                                   int32_t n_split) {
+  using Map = KlGradKMap<HI, DI>;
+  constexpr int KT = Map::KT, DPT = Map::DPT, NDG = Map::NDG, KPT = Map::KPT;
+  extern __shared__ __align__(16) float kl_k_smem[];
+  float (*qv)[DI] = reinterpret_cast<float (*)[DI]>(kl_k_smem);          // q^ of the current row
+  float (*a_s)[KT] = reinterpret_cast<float (*)[KT]>(kl_k_smem + HI * DI); // g w [x > 0]
+  float* g_s = kl_k_smem + HI * DI + HI * KT;                             // g[t, s] of the tile
+  unsigned long long* m_s =                                               // their sign masks
+      reinterpret_cast<unsigned long long*>(kl_k_smem + HI * DI + HI * KT + KT);
+  const int tile = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
   const int s0 = tile * KT;
-  const int k = threadIdx.x / NDG, dg = threadIdx.x % NDG;
-  const int s = s0 + k;
+  const int kg = threadIdx.x / NDG, dg = threadIdx.x % NDG;
   const int kvl = min(p.kv_len ? p.kv_len[b] : p.n_kv, p.n_kv);
   const int pos0 = p.q_pos0 ? p.q_pos0[b] : 0;
-  float acc[DG];
+  const int r_lo = static_cast<int>((static_cast<int64_t>(p.rows) * split) / n_split);
+  const int r_hi = static_cast<int>((static_cast<int64_t>(p.rows) * (split + 1)) / n_split);
+  float acc[KPT][DPT];
 #pragma unroll
-  for (int c = 0; c < DG; ++c) acc[c] = 0.f;
-  for (int r = 0; r < p.rows; ++r) {
+  for (int kk = 0; kk < KPT; ++kk)
+#pragma unroll
+    for (int c = 0; c < DPT; ++c) acc[kk][c] = 0.f;
+  for (int r = r_lo; r < r_hi; ++r) {
     const int t = p.row_begin + r;
     const int pos = pos0 + t;
     if (pos < s0 || s0 >= kvl) continue;   // no key of the tile is visible to this row (uniform)
@@ -483,21 +501,47 @@ __global__ void __launch_bounds__(kKlGradThreads) kl_grad_k_kernel(KlGradParams 
     }
     __syncthreads();
     for (int i = threadIdx.x; i < KT * HI; i += kKlGradThreads) {
-      const int kk = i / HI, j = i % HI;
-      a_s[kk][j] = ((m_s[kk] >> j) & 1ull) ? g_s[kk] * p.w[qrow * HI + j] : 0.f;
+      const int j = i / KT, kk = i % KT;
+      a_s[j][kk] = ((m_s[kk] >> j) & 1ull) ? g_s[kk] * p.w[qrow * HI + j] : 0.f;
     }
     __syncthreads();
-#pragma unroll 4
+#pragma unroll 2
     for (int j = 0; j < HI; ++j) {
-      const float a = a_s[k][j];
+      float qd[DPT], av[KPT];
 #pragma unroll
-      for (int c = 0; c < DG; ++c) acc[c] = fmaf(a, qv[j][dg * DG + c], acc[c]);
+      for (int c = 0; c < DPT; c += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(&qv[j][dg * DPT + c]);
+        qd[c] = v.x; qd[c + 1] = v.y; qd[c + 2] = v.z; qd[c + 3] = v.w;
+      }
+#pragma unroll
+      for (int kk = 0; kk < KPT; ++kk) av[kk] = a_s[j][kg * KPT + kk];
+#pragma unroll
+      for (int kk = 0; kk < KPT; ++kk)
+#pragma unroll
+        for (int c = 0; c < DPT; ++c) acc[kk][c] = fmaf(av[kk], qd[c], acc[kk][c]);
     }
   }
-  if (s < p.n_kv) {
-    float* dst = p.dk + (static_cast<size_t>(b) * p.n_kv + s) * DI + dg * DG;
+  // part[split, b, s, :] (the reduce kernel reads only keys < n_kv)
 #pragma unroll
-    for (int c = 0; c < DG; ++c) dst[c] += acc[c];
+  for (int kk = 0; kk < KPT; ++kk) {
+    const int s = s0 + kg * KPT + kk;
+    if (s < p.n_kv) {
+      float* dst = part + ((static_cast<size_t>(split) * gridDim.z + b) * p.n_kv + s) * DI + dg * DPT;
+#pragma unroll
+      for (int c = 0; c < DPT; c += 4)
+        *reinterpret_cast<float4*>(dst + c) =
+            make_float4(acc[kk][c], acc[kk][c + 1], acc[kk][c + 2], acc[kk][c + 3]);
+    }
+  }
+}
+
+// dk[i] += sum over splits (in order) of part[split, i], i over B * n_kv * DI.
+__global__ void kl_grad_k_reduce_kernel(const float* part, float* dk, int64_t n, int32_t n_split) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float v = dk[i];
+    for (int sp = 0; sp < n_split; ++sp) v += part[sp * n + i];
+    dk[i] = v;
   }
 }
 

@@ -53,3 +53,12 @@ def test_sampled_oracle_rows_are_evenly_spaced_and_distinct():
         rows = bench.oracle_sample_rows(cfg, n, off)
         assert len(rows) == n and rows.min() >= 0 and rows.max() < cfg.n_q
         assert (abs((rows[1:] - rows[:-1]) - cfg.n_q / n) <= 1).all()
+
+
+def test_warmup_loss_flops():
+    cfg = inputs.CONFIGS["prefill_4k"]
+    pairs = 4096 * 4097 // 2
+    fl = bench.warmup_loss_flops(cfg)
+    assert fl["probs_bf16"] == 2.0 * 128 * 576 * pairs
+    assert fl["scores_fp8"] == 2.0 * 64 * 128 * pairs
+    assert fl["grads_fp32"] == 2 * fl["scores_fp8"]
