@@ -56,6 +56,8 @@ def parse_args():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--shard", action="store_true",
                     help="run the query-sharded prefill path even on one rank")
+    ap.add_argument("--only-warmup-loss", action="store_true",
+                    help="time only the indexer warm-up loss + gradient on --workload")
     return ap.parse_args()
 
 
@@ -397,8 +399,8 @@ def breakdown(step, steps):
 # q read once plus out and lse written once (the latent gathers hit L2), so it
 # grows in proportion to the rows and is scaled by them. When the source no
 # longer matches, the figure is stale and the line reports null.
-ATTN_TRAFFIC_4K = {"bytes": 642.484736e6 + 1022.602e6, "rows": 4096,
-                   "source_sha256": "fc29016b7b6d77133fd629c9c6d3f7a7b7751e164c765ab4709e0c1e29010395"}
+ATTN_TRAFFIC_4K = {"bytes": 643.625984e6 + 1022.523e6, "rows": 4096,
+                   "source_sha256": "7c324e231f659fcf1a6ae1fd6917c248f049bb5435d29a7648b89ac8025802ce"}
 
 
 def kernel_source_sha256(name):
@@ -699,6 +701,13 @@ def main():
         dist = tdist
     peaks = measured_peaks()
     cfg = inputs.CONFIGS[args.workload]
+    if args.only_warmup_loss:
+        leg = warmup_loss_leg(cfg, 1000 + rank, args.steps, args.warmup)
+        if rank == 0:
+            print(json.dumps({"workload": cfg.name, "warmup_loss": leg}), flush=True)
+        if dist:
+            dist.destroy_process_group()
+        return
     # Several GPUs split ONE prefill by query rows (strong scaling): every
     # rank draws the same inputs and takes its share of the rows. --shard
     # runs that path on a single rank too.
