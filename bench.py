@@ -533,66 +533,106 @@ def decode_leg(cfg, seed, steps, warmup, dist, peaks):
 
 # ---------------------------------------------------------------- e2e
 
-def e2e(cfg, seed, steps, dist, shard=None):
-    """Same path through the public dsa_forward call with HOST buffers:
-    every step copies the inputs host->device from pinned memory, runs the
-    forward and reads the result (out, lse, indices) back. Sharded: each
-    rank copies its rows' query inputs and its slice of the keys, the keys
-    are all-gathered on the GPUs, and each rank reads back its rows."""
+def e2e(cfg, seed, steps, dist, shard=None, n_chunks=8):
+    """The same path through the public dsa_forward_ex call with HOST
+    buffers: every step copies the inputs host->device from pinned memory,
+    runs the forward and reads the results (out, lse, indices) back.
+
+    The copies are pipelined against the compute: the rows (this rank's rows
+    when sharded) are cut into n_chunks runs of consecutive 4-row groups;
+    chunk c's query inputs go up on a copy stream, its forward runs on a
+    compute stream (dsa_forward_ex with the chunk's absolute row positions,
+    against all keys, which go up first), and its results come down on a
+    third stream, so the host link in both directions overlaps the kernels.
+    Sharded: each rank uploads its slice of the keys and all-gathers them."""
     import torch
     import sparse_attention_long_fp8_b200 as dsa
     from sparse_attention_long_fp8_b200 import inputs, shard as shard_mod
     dev_inp = dsa.make_inputs(cfg, seed=seed, device="cuda")
-    layout, kslice, full_n_kv = None, None, cfg.n_kv
+    full_n_kv = cfg.n_kv
+    if cfg.batch != 1:
+        raise ValueError("the pipelined e2e splits the rows of one sequence")
+    rows_all = (shard_mod.shard_rows(cfg.n_q, shard[1], shard[0]) if shard is not None
+                else None)
+    kslice = None
     if shard is not None:
-        rank, ranks = shard
-        rows = shard_mod.shard_rows(cfg.n_q, ranks, rank)
-        dev_inp = shard_mod.shard_inputs(dev_inp, rows)
-        cfg = inputs.custom_config(cfg.name, n_q=len(rows), name=f"{cfg.name}_shard{rank}")
+        dev_inp = shard_mod.shard_inputs(dev_inp, rows_all)
         if dist is not None:
-            kslice = shard_mod.key_slice(cfg.n_kv, ranks, rank)
-    qkeys = ["q_fp8", "q_scale", "w", "q_pos0", "kv_len", "q"] + (["row_pos"] if shard else [])
+            kslice = shard_mod.key_slice(full_n_kv, shard[1], shard[0])
+    else:
+        dev_inp["row_pos"] = (dev_inp["q_pos0"][:, None] +
+                              torch.arange(cfg.n_q, device="cuda", dtype=torch.int32)[None, :])
+    T = dev_inp["q"].shape[1]
+    qkeys = ["q_fp8", "q_scale", "w", "q", "row_pos"]
     kkeys = ["k_fp8", "k_scale", "kv"]
-    host = {}
-    for k in qkeys + kkeys:
+    host, dev = {}, {}
+    for k in qkeys + kkeys + ["kv_len", "q_pos0"]:
         t = dev_inp[k]
         if kslice is not None and k in kkeys:
             t = t[:, kslice[0]:kslice[1]]
         host[k] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
         host[k].copy_(t)
-    dev = {k: torch.empty_like(dev_inp[k]) for k in qkeys + kkeys}
+        dev[k] = torch.empty_like(dev_inp[k])
     dev_local = ({k: torch.empty(host[k].shape, dtype=host[k].dtype, device="cuda") for k in kkeys}
                  if kslice is not None else None)
     del dev_inp
-    if shard is not None:
-        layout = dsa.make_layout(row_pos=dev["row_pos"])
-    shape = dsa.shape_of(cfg)
-    B, T = cfg.batch, cfg.n_q
-    out = torch.empty(B, T, cfg.heads, cfg.v_dim, device="cuda")
-    lse = torch.empty(B, T, cfg.heads, device="cuda")
-    idx = torch.empty(B, T, cfg.topk, dtype=torch.int32, device="cuda")
+    # chunks: runs of whole 4-row groups
+    groups = (T + 3) // 4
+    bounds = [min(T, 4 * ((groups * c) // n_chunks)) for c in range(n_chunks + 1)]
+    chunks = [(bounds[c], bounds[c + 1]) for c in range(n_chunks) if bounds[c + 1] > bounds[c]]
+    out = torch.empty(1, T, cfg.heads, cfg.v_dim, device="cuda")
+    lse = torch.empty(1, T, cfg.heads, device="cuda")
+    idx = torch.empty(1, T, cfg.topk, dtype=torch.int32, device="cuda")
     h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     h_lse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     h_idx = torch.empty(idx.shape, dtype=idx.dtype, pin_memory=True)
-    ws, n = dsa.alloc_workspace(shape, dsa.DSA_OP_FORWARD)
+    plans = []
+    for r0, r1 in chunks:
+        ccfg = inputs.custom_config(cfg.name, n_q=r1 - r0, n_kv=full_n_kv, name="e2e_chunk")
+        shape = dsa.shape_of(ccfg)
+        ws, n = dsa.alloc_workspace(shape, dsa.DSA_OP_FORWARD)
+        lay = dsa.make_layout(row_pos=dev["row_pos"][:, r0:r1])
+        plans.append((r0, r1, shape, ws, n, lay))
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in (h_out, h_lse, h_idx))
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
 
     def one():
-        for k in qkeys:
-            dev[k].copy_(host[k], non_blocking=True)
-        for k in kkeys:
-            if dev_local is None:
-                dev[k].copy_(host[k], non_blocking=True)
-            else:
-                dev_local[k].copy_(host[k], non_blocking=True)
-                dev[k].copy_(shard_mod.all_gather_keys(dev_local[k], full_n_kv, dist))
-        dsa.dsa_forward(shape, dev["q_fp8"], dev["q_scale"], dev["w"], dev["k_fp8"],
-                        dev["k_scale"], dev["q_pos0"], dev["kv_len"], dev["q"], dev["kv"], idx,
-                        out, lse, ws, n, layout=layout)
-        h_out.copy_(out, non_blocking=True)
-        h_lse.copy_(lse, non_blocking=True)
-        h_idx.copy_(idx, non_blocking=True)
+        cur = torch.cuda.current_stream()
+        s_in.wait_stream(cur)
+        with torch.cuda.stream(s_in):
+            for k in kkeys + ["kv_len", "q_pos0"]:
+                (dev_local[k] if dev_local is not None and k in kkeys else dev[k]).copy_(
+                    host[k], non_blocking=True)
+            keys_in = torch.cuda.Event()
+            keys_in.record(s_in)
+        s_comp.wait_event(keys_in)
+        if dev_local is not None:
+            with torch.cuda.stream(s_comp):
+                for k in kkeys:
+                    dev[k].copy_(shard_mod.all_gather_keys(dev_local[k], full_n_kv, dist))
+        for r0, r1, shape, ws, n, lay in plans:
+            with torch.cuda.stream(s_in):
+                for k in qkeys:
+                    dev[k][:, r0:r1].copy_(host[k][:, r0:r1], non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(s_in)
+            s_comp.wait_event(ready)
+            with torch.cuda.stream(s_comp):
+                dsa.dsa_forward(shape, dev["q_fp8"][:, r0:r1], dev["q_scale"][:, r0:r1],
+                                dev["w"][:, r0:r1], dev["k_fp8"], dev["k_scale"], dev["q_pos0"],
+                                dev["kv_len"], dev["q"][:, r0:r1], dev["kv"], idx[:, r0:r1],
+                                out[:, r0:r1], lse[:, r0:r1], ws, n, stream=s_comp, layout=lay)
+                done = torch.cuda.Event()
+                done.record(s_comp)
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                h_out[:, r0:r1].copy_(out[:, r0:r1], non_blocking=True)
+                h_lse[:, r0:r1].copy_(lse[:, r0:r1], non_blocking=True)
+                h_idx[:, r0:r1].copy_(idx[:, r0:r1], non_blocking=True)
+        cur.wait_stream(s_out)
+        cur.wait_stream(s_comp)
+        cur.wait_stream(s_in)
 
     one()
     torch.cuda.synchronize()
@@ -608,7 +648,7 @@ def e2e(cfg, seed, steps, dist, shard=None):
     torch.cuda.synchronize()
     dsa.dsa_check()
     ms = max_over_ranks(s.elapsed_time(e) / steps, dist)
-    del host, dev, out, lse, idx, h_out, h_lse, h_idx, ws, dev_local
+    del host, dev, out, lse, idx, h_out, h_lse, h_idx, plans, dev_local
     torch.cuda.empty_cache()
     return ms, h2d, d2h
 
