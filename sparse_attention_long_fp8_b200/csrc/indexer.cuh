@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(IndexerTile<HI, DI, QG>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n_compute > 0) {
+    if (n_compute > 0 && elect_one()) {
       constexpr uint32_t idesc = umma_idesc(T::M, T::N, 0u, 0u, 0u, 0u);
       bool ok = mbar_wait(q_full, 0);
       const uint32_t q_addr = smem_u32(q_smem);

@@ -159,27 +159,27 @@ __global__ void __launch_bounds__(288, 1) kl_probs_kernel(KlProbParams p) {
     cp_async_wait_all();
   } else if (warp == 4) {
     // ------------------------------------------------------------ S = Q C^T issuer
-    constexpr uint32_t idesc = umma_idesc(128, NK, 1u, 1u, 0u, 0u);
-    const uint64_t c_desc0 = umma_desc(smem_u32(c_smem), 16, 1024, 2);
-    bool ok = mbar_wait(q_ready, 0);
-    tc_fence_after();
-    for (int i = 0; i < n_it && ok; ++i) {
-      const int st = i & 1;
-      ok = mbar_wait(&c_full[st], (i >> 1) & 1) && mbar_wait(&s_free[st], ((i >> 1) & 1) ^ 1);
-      if (!ok) break;
-      fence_proxy_async_smem();
+    // one elected lane runs the whole loop (see elect_one)
+    if (elect_one()) {
+      constexpr uint32_t idesc = umma_idesc(128, NK, 1u, 1u, 0u, 0u);
+      const uint64_t c_desc0 = umma_desc(smem_u32(c_smem), 16, 1024, 2);
+      bool ok = mbar_wait(q_ready, 0);
       tc_fence_after();
-      const uint32_t d_s = tmem_base + T::COL_S + st * NK;
-      const uint64_t cd = c_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
+      for (int i = 0; i < n_it && ok; ++i) {
+        const int st = i & 1;
+        ok = mbar_wait(&c_full[st], (i >> 1) & 1) && mbar_wait(&s_free[st], ((i >> 1) & 1) ^ 1);
+        if (!ok) break;
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint32_t d_s = tmem_base + T::COL_S + st * NK;
+        const uint64_t cd = c_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
 #pragma unroll
-      for (int db = 0; db < T::NDB; ++db)
+        for (int db = 0; db < T::NDB; ++db)
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = cd + ((db * T::DB_BYTES + kk * 32) >> 4);
-          if (elect_one())
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = cd + ((db * T::DB_BYTES + kk * 32) >> 4);
             umma_bf16_ts(d_s, tmem_base + T::COL_Q + db * 32 + kk * 8, bd, idesc, (db | kk) ? 1u : 0u);
-        }
-      if (elect_one()) {
+          }
         umma_commit(&c_empty[st]);
         umma_commit(&s_full[st]);
       }

@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(IndexerTopkTile<HI, DI, QG>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (n_compute > 0) {
+    if (n_compute > 0 && elect_one()) {   // one lane runs the whole loop (see elect_one)
       constexpr uint32_t idesc = umma_idesc(T::M, T::N, 0u, 0u, 0u, 0u);
       const uint64_t q_desc = umma_desc(smem_u32(q_smem), 16, T::SBO, T::SWIZZLE);
       const uint64_t k_desc0 = umma_desc(smem_u32(k_smem), 16, T::SBO, T::SWIZZLE);
@@ -537,13 +537,10 @@ __global__ void __launch_bounds__(IndexerTopkTile<HI, DI, QG>::THREADS, 1)
         const uint64_t kd = k_desc0 + static_cast<uint32_t>(st * (T::K_BYTES >> 4));
 #pragma unroll
         for (int kk = 0; kk < DI / 32; ++kk)
-          if (elect_one())
-            umma_f8_ss(tmem_base + buf * T::N, kd + ((kk * 32) >> 4), q_desc + ((kk * 32) >> 4),
-                       idesc, kk > 0 ? 1u : 0u);
-        if (elect_one()) {
-          umma_commit(&k_empty[st]);
-          umma_commit(&acc_full[buf]);
-        }
+          umma_f8_ss(tmem_base + buf * T::N, kd + ((kk * 32) >> 4), q_desc + ((kk * 32) >> 4),
+                     idesc, kk > 0 ? 1u : 0u);
+        umma_commit(&k_empty[st]);
+        umma_commit(&acc_full[buf]);
       }
     }
     __syncwarp();

@@ -38,6 +38,13 @@ __device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ void sts_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                       uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
 // The first 1024-byte aligned byte of a dynamic shared-memory array. The
 // offset is computed from the shared-window address and applied to the array
 // pointer itself, so the compiler still knows the result points to shared
@@ -58,10 +65,10 @@ __device__ __forceinline__ void raise_error(unsigned int code) {
 }
 
 // True in exactly one lane of a converged warp (the lowest active lane, so
-// always the same thread when the whole warp is active). Single-thread
-// instructions (tcgen05.mma, tcgen05.commit) issued under it from warp-uniform
-// control flow keep their operands in the uniform datapath; issuing them from
-// an `if (lane == 0)` branch costs measurably more issue slots per MMA.
+// always the same thread when the whole warp is active). An MMA issuer elects
+// once and lets that lane run its whole loop: an elect (or a lane test) per
+// tcgen05.mma costs more issue time than an M = 128, N = 64 MMA takes to run
+// (measured on B200: 64 against 32 cycles per MMA with A in TMEM).
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred;
   asm volatile("{ .reg .pred p; elect.sync _|p, 0xffffffff; selp.u32 %0, 1, 0, p; }"
@@ -310,6 +317,27 @@ __device__ __forceinline__ void cp_async_wait_all() {
 // Named barrier for a subset of warps (ids 1..15; 0 is __syncthreads).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Named barrier over `nthreads` threads that also returns the AND of every
+// participant's `pred` (so that the participants leave a loop together).
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.and.pred q, %2, %3, p;"
+      " selp.u32 %0, 1, 0, q; }"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+// 2^x by the hardware approximation (PTX ex2.approx.ftz: relative error
+// about 2^-22; -inf gives +0, results below 2^-126 flush to zero).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 }  // namespace dsa

@@ -7,9 +7,11 @@
 //   * gathers the full 1152-byte latent rows of the selected keys into a
 //     2-stage ring of 64-key blocks (cp.async, completion on mbarriers);
 //   * computes the complete logits S = Q C^T (128 heads x 64 keys per block):
-//     Q's five 64-dim blocks that only the logits use live in TMEM (A operand
-//     read from TMEM), its four V-half blocks in shared memory;
-//   * runs the online softmax and accumulates O for its 256 value dims.
+//     six of Q's nine 64-dim blocks live in TMEM (A operand read from TMEM),
+//     three in shared memory;
+//   * runs the online softmax and accumulates O for its 256 value dims. The
+//     two softmax warps of a TMEM lane quarter share each block's row maxima
+//     through shared memory and a named barrier.
 // The logits are computed twice per row (once per CTA) and the rows gathered
 // twice (L2 serves the second read); in exchange no partial result crosses
 // between SMs: on this part DSMEM stores move ~11 bytes per cycle per SM,
@@ -20,14 +22,15 @@
 // logit MMAs of a block run over the logit-only part first, so the gather of
 // block i + 2 overlaps S(i + 1) and PV(i).
 //
-// S is double-buffered in TMEM, and P(i) (bf16, 32 columns) is written over
-// the first half of S(i)'s own buffer once both softmax warps of a lane
-// quarter have read it. S(i + 1) is issued as soon as PV(i - 1) has released
-// its buffer, so the tensor pipe does not wait for the softmax to read S(i).
+// S has one TMEM buffer, released as soon as the eight softmax warps have
+// loaded it into registers; P(i) (bf16) goes to one of two shared-memory
+// buffers and the PV MMA reads it from there. So S(i + 1) waits only for the
+// load of S(i), not for the softmax or PV(i), and the tensor pipe runs PV(i)
+// in the gap between S(i + 1) and S(i + 2).
 //
-// TMEM per CTA: O 256 columns, S 2 x 64, Q 128 (four logit-only dim blocks)
-// = 512. Q's other five dim blocks (the V half and the RoPE block) are in
-// shared memory.
+// TMEM per CTA: O 256 columns, S 64, Q 192 (six 64-dim blocks: the five that
+// only the logits read and the first of the V half) = 512. Q's other three
+// V-half blocks are in shared memory.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -49,33 +52,41 @@ struct VhTile {
   static constexpr int DB_BYTES = NK * 128;     // one 64-dim block of a stage
   static constexpr int STAGE_BYTES = NDB * DB_BYTES;
   static constexpr int STAGES = 2;
-  static constexpr int XT = 4;                  // logit-only Q blocks held in TMEM
-  static constexpr int QSB = VDB + 1;           // Q blocks in shared memory: V half + RoPE
+  static constexpr int XT = 6;                  // Q blocks held in TMEM
+  static constexpr int QSB = NDB - XT;          // Q blocks in shared memory (V half 1..3)
   static constexpr int QS_BYTES = QSB * M * 128;
+  static constexpr int P_BYTES = M * NK * 2;    // one bf16 P tile, K-major 128-byte swizzle
   static constexpr int PRODUCERS = 128;
   static constexpr int THREADS = 448;           // gather 0-3, S MMA 4, softmax 5-12, PV MMA 13
   static constexpr int SOFTMAX_WARPS = 8;       // two per TMEM lane quarter, 32 keys each
-  static constexpr int COL_O = 0, COL_S = 256, COL_Q = 384;   // S buffer b at COL_S + 64 b
+  static constexpr int COL_O = 0, COL_S = 256, COL_Q = 320;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int OFF_C = 0;
   static constexpr int OFF_QS = STAGES * STAGE_BYTES;
-  static constexpr int OFF_RED = OFF_QS + QS_BYTES;          // [2 parity][2 halves][128] fp32
+  static constexpr int OFF_P = OFF_QS + QS_BYTES;            // [2] P tiles
+  static constexpr int OFF_RED = OFF_P + 2 * P_BYTES;        // [2 parity][2 halves][128] fp32
   static constexpr int OFF_END = OFF_C;      // [half][l, l_mma][128] fp32, after the last PV
+  static constexpr int OFF_OSTAGE = OFF_C + 4096;            // O rows on their way out
   static constexpr int OFF_BAR = OFF_RED + 2 * 2 * M * 4;
-  static constexpr int NUM_BARS = 4 * STAGES + 6 + 8 + 4;    // stages, singles, red[8], end[4]
+  static constexpr int NUM_BARS = 4 * STAGES + 7 + 4;        // stages, singles, end[4]
   // No alignment slack: the dynamic shared memory of this kernel starts on a
   // 1024-byte boundary (checked at run time; a misaligned base is reported).
   static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16;
   static_assert(SMEM_BYTES <= 232448, "shared memory");
-  static_assert(STAGE_BYTES % 1024 == 0 && OFF_QS % 1024 == 0, "1024-byte aligned operands");
-  static_assert(COL_Q + XT * 32 == 512, "TMEM columns");
+  static_assert(STAGE_BYTES % 1024 == 0 && OFF_QS % 1024 == 0 && OFF_P % 1024 == 0,
+                "1024-byte aligned operands");
+  static_assert(COL_S + NK == COL_Q && COL_Q + XT * 32 == 512, "TMEM columns");
+  static_assert(OFF_OSTAGE + M * VH * 4 <= OFF_QS, "O staging fits in the stage area");
 };
 
-// Latent dim block of the t-th Q block held in TMEM (t = 0..3): the other
-// half's four value blocks. The u-th Q block in shared memory (u = 0..4) is
-// block 4v + u of this CTA's value half, then the RoPE block 8.
-__device__ __forceinline__ int vh_tblock(int t, int v) { return t + 4 * (1 - v); }
-__device__ __forceinline__ int vh_sblock(int u, int v) { return u == 4 ? 8 : 4 * v + u; }
+// Latent dim block of the t-th Q block held in TMEM (t = 0..5): the other
+// half's four value blocks, the RoPE block 8, then block 4v (the first of this
+// CTA's value half). The u-th Q block in shared memory (u = 0..2) is block
+// 4v + 1 + u.
+__device__ __forceinline__ int vh_tblock(int t, int v) {
+  return t < 4 ? t + 4 * (1 - v) : (t == 4 ? 8 : 4 * v);
+}
+__device__ __forceinline__ int vh_sblock(int u, int v) { return 4 * v + 1 + u; }
 
 // Warp roles: 0-3 gather (cp.async, 16 bytes per copy); 4 issues
 // the logit MMAs and owns TMEM; 5-12 run the softmax (two warps per TMEM lane
@@ -93,12 +104,12 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
   uint64_t* cv_full = bars + T::STAGES;          // [2] V-half blocks landed
   uint64_t* cx_empty = bars + 2 * T::STAGES;     // [2] S of the stage's block finished
   uint64_t* cv_empty = bars + 3 * T::STAGES;     // [2] PV of the stage's block finished
-  uint64_t* s_full = bars + 4 * T::STAGES;       // [2] S tile of buffer b written
-  uint64_t* pv_done = s_full + 2;                // [2] PV of buffer b finished (buffer free, O updated)
-  uint64_t* p_full = s_full + 4;                 // P tile written
-  uint64_t* q_ready = s_full + 5;                // Q in TMEM and shared memory
-  uint64_t* red_bar = s_full + 6;                // [parity][quarter]: both half maxima written
-  uint64_t* end_bar = s_full + 14;               // [quarter]: both halves of l, l_mma written
+  uint64_t* s_full = bars + 4 * T::STAGES;       // S tile written
+  uint64_t* s_free = s_full + 1;                 // S tile loaded by all softmax warps
+  uint64_t* p_full = s_full + 2;                 // [2] P tile of buffer b written
+  uint64_t* pv_done = s_full + 4;                // [2] PV of buffer b finished (buffer free, O updated)
+  uint64_t* q_ready = s_full + 6;                // Q in TMEM and shared memory
+  uint64_t* end_bar = s_full + 7;                // [quarter]: both halves of l, l_mma written
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + T::NUM_BARS);
 
   if ((smem_u32(smem_raw) & 1023u) != 0) {      // see SMEM_BYTES: no slack to realign
@@ -124,13 +135,14 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
       mbar_init(&cx_empty[s], 1);
       mbar_init(&cv_empty[s], 1);
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, T::SOFTMAX_WARPS);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], T::SOFTMAX_WARPS);
       mbar_init(&pv_done[s], 1);
     }
-    mbar_init(p_full, T::SOFTMAX_WARPS);
     mbar_init(q_ready, T::SOFTMAX_WARPS);
-    for (int s = 0; s < 12; ++s) mbar_init(&red_bar[s], 2);
+    for (int s = 0; s < 4; ++s) mbar_init(&end_bar[s], 2);
     fence_mbar_init();
   }
   if (warp == 4) {
@@ -206,82 +218,85 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
     cp_async_wait_all();
   } else if (warp == 4) {
     // ------------------------------------------------------------ S = Q C^T issuer
-    // The whole warp runs the loop; one elected lane issues. Descriptors are
-    // formed once: adding (byte offset >> 4) to a descriptor moves its start
-    // address (every shared address here is below 256 KB, so the 14-bit
-    // field cannot carry).
-    constexpr uint32_t idesc_s = umma_idesc(128, NK, 1u, 1u, 0u, 0u);
-    const uint64_t c_desc0 = umma_desc(smem_u32(c_smem), 16, 1024, 2);
-    const uint64_t q_desc0 = umma_desc(smem_u32(qs_smem), 16, 1024, 2);
-    const uint32_t x_shift = static_cast<uint32_t>(4 * (1 - vh) * T::DB_BYTES) >> 4;
-    const uint32_t v_shift = static_cast<uint32_t>(4 * vh * T::DB_BYTES) >> 4;
-    bool ok = mbar_wait(q_ready, 0);
-    tc_fence_after();
-    for (int i = 0; i < n_blocks && ok; ++i) {
-      const int st = i % T::STAGES;
-      const uint32_t ph = (i / T::STAGES) & 1;
-      const int sb = i & 1;                            // S buffer of block i
-      // buffer sb is free once PV(i - 2) has read the P it held
-      ok = mbar_wait(&pv_done[sb], ((i >> 1) & 1) ^ 1) && mbar_wait(&cx_full[st], ph);
-      if (!ok) break;
-      fence_proxy_async_smem();
+    // One elected lane runs the whole loop: an elect per instruction costs
+    // more issue time than an N = 64 MMA takes to execute (measured: 64
+    // against 32 cycles per MMA with A in TMEM). Descriptors are formed once:
+    // adding (byte offset >> 4) to a descriptor moves its start address
+    // (every shared address here is below 256 KB, so the 14-bit field cannot
+    // carry).
+    if (elect_one()) {
+      constexpr uint32_t idesc_s = umma_idesc(128, NK, 1u, 1u, 0u, 0u);
+      const uint64_t c_desc0 = umma_desc(smem_u32(c_smem), 16, 1024, 2);
+      const uint64_t q_desc0 = umma_desc(smem_u32(qs_smem), 16, 1024, 2);
+      const uint32_t x_shift = static_cast<uint32_t>(4 * (1 - vh) * T::DB_BYTES) >> 4;
+      const uint32_t v_shift = static_cast<uint32_t>(4 * vh * T::DB_BYTES) >> 4;
+      const uint32_t d_s = tmem_base + T::COL_S;
+      bool ok = mbar_wait(q_ready, 0);
       tc_fence_after();
-      const uint32_t d_s = tmem_base + T::COL_S + sb * T::NK;
-      const uint64_t cd = c_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
-      // logit-only part of the stage: the other half's value blocks with Q
-      // from TMEM, then the RoPE block with Q from shared memory
+      for (int i = 0; i < n_blocks && ok; ++i) {
+        const int st = i % T::STAGES;
+        const uint32_t ph = (i / T::STAGES) & 1;
+        // the S buffer is free once every softmax warp has loaded S(i - 1)
+        ok = (i == 0 || mbar_wait(s_free, (i - 1) & 1)) && mbar_wait(&cx_full[st], ph);
+        if (!ok) break;
+        fence_proxy_async_smem();
+        tc_fence_after();
+        const uint64_t cd = c_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
+        // logit-only part of the stage (the other half's value blocks, then
+        // the RoPE block), Q from TMEM
 #pragma unroll
-      for (int t = 0; t < T::XT; ++t)
+        for (int t = 0; t < T::XDB; ++t)
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = cd + x_shift + ((t * T::DB_BYTES + kk * 32) >> 4);
-          if (elect_one())
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t off = (t < 4 ? t * T::DB_BYTES : 8 * T::DB_BYTES) + kk * 32;
+            const uint64_t bd = cd + (t < 4 ? x_shift : 0u) + (off >> 4);
             umma_bf16_ts(d_s, tmem_base + T::COL_Q + t * 32 + kk * 8, bd, idesc_s,
                          (t | kk) ? 1u : 0u);
-        }
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = q_desc0 + ((4 * T::M * 128 + kk * 32) >> 4);
-        const uint64_t bd = cd + ((8 * T::DB_BYTES + kk * 32) >> 4);
-        if (elect_one()) umma_bf16_ss(d_s, ad, bd, idesc_s, 1u);
-      }
-      if (elect_one()) umma_commit(&cx_empty[st]);
-      ok = mbar_wait(&cv_full[st], ph);
-      if (!ok) break;
-      fence_proxy_async_smem();
-      tc_fence_after();
-      // V-half blocks, Q from shared memory
-#pragma unroll
-      for (int u = 0; u < T::VDB; ++u)
+          }
+        umma_commit(&cx_empty[st]);
+        ok = mbar_wait(&cv_full[st], ph);
+        if (!ok) break;
+        fence_proxy_async_smem();
+        tc_fence_after();
+        // V-half blocks: the first with Q from TMEM, the other three from
+        // shared memory
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = q_desc0 + ((u * T::M * 128 + kk * 32) >> 4);
-          const uint64_t bd = cd + v_shift + ((u * T::DB_BYTES + kk * 32) >> 4);
-          if (elect_one()) umma_bf16_ss(d_s, ad, bd, idesc_s, 1u);
+          const uint64_t bd = cd + v_shift + ((kk * 32) >> 4);
+          umma_bf16_ts(d_s, tmem_base + T::COL_Q + T::XDB * 32 + kk * 8, bd, idesc_s, 1u);
         }
-      if (elect_one()) umma_commit(&s_full[sb]);
+#pragma unroll
+        for (int u = 0; u < T::QSB; ++u)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = q_desc0 + ((u * T::M * 128 + kk * 32) >> 4);
+            const uint64_t bd = cd + v_shift + (((u + 1) * T::DB_BYTES + kk * 32) >> 4);
+            umma_bf16_ss(d_s, ad, bd, idesc_s, 1u);
+          }
+        umma_commit(s_full);
+      }
     }
     __syncwarp();
   } else if (warp == 13) {
     // ------------------------------------------------------------ O += P V issuer
-    constexpr uint32_t idesc_pv = umma_idesc(128, T::VH, 1u, 1u, 0u, 1u);
-    const uint64_t v_desc0 =
-        umma_desc(smem_u32(c_smem) + 4 * vh * T::DB_BYTES, T::DB_BYTES, 1024, 2);
-    for (int j = 0; j < n_blocks; ++j) {
-      const int st = j % T::STAGES;
-      if (!mbar_wait(p_full, j & 1)) break;
-      tc_fence_after();
-      // P(j) exists only after S(j) was read, so S(j) has completed: when
-      // PV(j) completes, both readers of the V-half blocks are done, and the
-      // S / P buffer of block j is free.
-      const uint64_t vd = v_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
-      const uint32_t a_p = tmem_base + T::COL_S + (j & 1) * T::NK;   // P over S's first half
+    // P(j) exists only after S(j) was read, so S(j) has completed: when PV(j)
+    // completes, both readers of the V-half blocks are done, and P buffer
+    // j & 1 is free. One elected lane issues (as for S).
+    if (elect_one()) {
+      constexpr uint32_t idesc_pv = umma_idesc(128, T::VH, 1u, 1u, 0u, 1u);
+      const uint64_t v_desc0 =
+          umma_desc(smem_u32(c_smem) + 4 * vh * T::DB_BYTES, T::DB_BYTES, 1024, 2);
+      const uint64_t p_desc0 = umma_desc(smem_u32(smem + T::OFF_P), 16, 1024, 2);
+      for (int j = 0; j < n_blocks; ++j) {
+        const int st = j % T::STAGES;
+        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1)) break;
+        tc_fence_after();
+        const uint64_t vd = v_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
+        const uint64_t pd = p_desc0 + static_cast<uint32_t>((j & 1) * (T::P_BYTES >> 4));
 #pragma unroll
-      for (int kk = 0; kk < NK / 16; ++kk)
-        if (elect_one())
-          umma_bf16_ts(tmem_base + T::COL_O, a_p + kk * 8, vd + ((kk * 2048) >> 4), idesc_pv,
-                       (j > 0 || kk > 0) ? 1u : 0u);
-      if (elect_one()) {
+        for (int kk = 0; kk < NK / 16; ++kk)
+          umma_bf16_ss(tmem_base + T::COL_O, pd + ((kk * 32) >> 4), vd + ((kk * 2048) >> 4),
+                       idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&cv_empty[st]);
         umma_commit(&pv_done[j & 1]);
       }
@@ -295,30 +310,43 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
     float* red = reinterpret_cast<float*>(smem + T::OFF_RED);   // [parity][half][128]
 
-    // Q into TMEM (four logit-only blocks; the two warps of a quarter take
-    // alternate 16-column chunks) and shared memory (V-half blocks and the
-    // RoPE block, K-major 128-byte swizzle; the two warps alternate blocks).
+    // Q into TMEM (six blocks; the two warps of a quarter take alternate
+    // 16-column chunks) and shared memory (three V-half blocks, K-major
+    // 128-byte swizzle; the two warps alternate blocks). The shared-memory
+    // part goes by cp.async, and every load of the TMEM part is issued before
+    // the first TMEM store, so the whole of Q costs one memory round trip.
     {
       const __nv_bfloat16* qh = p.q + (static_cast<size_t>(row) * p.H + min(h, p.H - 1)) * T::DQK;
       const bool live = h < p.H;
-      for (int c = half; c < T::XT * 2; c += 2) {
-        uint32_t v[16];
-        const uint4* src = reinterpret_cast<const uint4*>(qh + vh_tblock(c >> 1, vh) * 64 + (c & 1) * 32);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint4 u = live ? src[k] : make_uint4(0u, 0u, 0u, 0u);
-          v[4 * k] = u.x; v[4 * k + 1] = u.y; v[4 * k + 2] = u.z; v[4 * k + 3] = u.w;
-        }
-        tmem_st16(tmem_base + lane_addr + T::COL_Q + c * 16, v);
-      }
       for (int u = half; u < T::QSB; u += 2) {
-        const uint4* src = reinterpret_cast<const uint4*>(qh + vh_sblock(u, vh) * 64);
-        uint8_t* dst = qs_smem + u * (T::M * 128) + (h >> 3) * 1024 + (h & 7) * 128;
+        const __nv_bfloat16* src = qh + vh_sblock(u, vh) * 64;
+        const uint32_t dst = smem_u32(qs_smem) + u * (T::M * 128) + (h >> 3) * 1024 + (h & 7) * 128;
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch)
-          *reinterpret_cast<uint4*>(dst + ((ch ^ (h & 7)) << 4)) =
-              live ? src[ch] : make_uint4(0u, 0u, 0u, 0u);
+          cp_async_16(dst + ((ch ^ (h & 7)) << 4), src + ch * 8, live ? 16u : 0u);
       }
+      constexpr int NCH = T::XT;                 // TMEM chunks per warp (of 2 * XT)
+      uint4 qv[NCH][4];
+#pragma unroll
+      for (int k = 0; k < NCH; ++k) {
+        const int c = half + 2 * k;
+        const uint4* src =
+            reinterpret_cast<const uint4*>(qh + vh_tblock(c >> 1, vh) * 64 + (c & 1) * 32);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) qv[k][j] = live ? __ldg(src + j) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int k = 0; k < NCH; ++k) {
+        uint32_t v[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[4 * j] = qv[k][j].x; v[4 * j + 1] = qv[k][j].y;
+          v[4 * j + 2] = qv[k][j].z; v[4 * j + 3] = qv[k][j].w;
+        }
+        tmem_st16(tmem_base + lane_addr + T::COL_Q + (half + 2 * k) * 16, v);
+      }
+      cp_async_wait_all();
       fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
@@ -337,45 +365,52 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
     int idx_next = load_idx(0);
     uint32_t sr[32];
     float z[32];
-    for (int i = 0; i < n_blocks && ok; ++i) {
-      // ---- logits of this warp's 32 keys from S buffer i & 1
+    // this thread's row of a P tile: keys half * 32 .. + 31 are 16-byte chunks
+    // 4 half .. 4 half + 3 of a 128-byte row, stored at chunk c ^ (h & 7)
+    const uint32_t p_row = smem_u32(smem + T::OFF_P) + (h >> 3) * 1024 + (h & 7) * 128;
+    for (int i = 0; i < n_blocks; ++i) {
+      // ---- logits of this warp's 32 keys; the S buffer is released at once.
+      // A failed wait does not leave the loop before the partner exchange:
+      // the two warps of a quarter meet at a named barrier every block and
+      // leave together when either has failed.
       const int idx = idx_next;
       idx_next = load_idx(i + 1);
       const uint32_t vmask = __ballot_sync(0xffffffffu, idx >= 0 && idx < p.n_kv);
-      const uint32_t col_s = T::COL_S + (i & 1) * T::NK;
-      if (!(ok = mbar_wait(&s_full[i & 1], (i >> 1) & 1))) break;
+      if (ok) ok = mbar_wait(s_full, i & 1);
       tc_fence_after();
-      tmem_ld32(tmem_base + lane_addr + col_s + half * 32, sr);
+      tmem_ld32(tmem_base + lane_addr + T::COL_S + half * 32, sr);
       tmem_wait_ld();
-      // ---- block max over the 64 keys, shared with the partner warp
-      float hmax = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        z[j] = ((vmask >> j) & 1u) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
-        hmax = fmaxf(hmax, z[j]);
-      }
-      float* red_i = red + (i & 1) * (2 * T::M);
-      red_i[half * T::M + h] = hmax;
-      // After this exchange both warps of the quarter have read their S
-      // columns, so P may overwrite the buffer's first 32 columns.
       tc_fence_before();
       __syncwarp();
-      uint64_t* rb = &red_bar[(i & 1) * 4 + quarter];
-      if (lane == 0) mbar_arrive(rb);
-      if (!(ok = mbar_wait(rb, (i >> 1) & 1))) break;
-      tc_fence_after();
+      if (lane == 0) mbar_arrive(s_free);
+      // ---- block max over the 64 keys, shared with the partner warp
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        z[j] = ((vmask >> j) & 1u) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
+      float mx[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        mx[r] = fmaxf(fmaxf(fmaxf(z[r], z[r + 4]), fmaxf(z[r + 8], z[r + 12])),
+                      fmaxf(fmaxf(z[r + 16], z[r + 20]), fmaxf(z[r + 24], z[r + 28])));
+      const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      float* red_i = red + (i & 1) * (2 * T::M);
+      red_i[half * T::M + h] = hmax;
+      if (!named_bar_and(1u + static_cast<uint32_t>(quarter), 64u, ok)) {
+        ok = false;
+        break;
+      }
       const float bmax = fmaxf(hmax, red_i[(half ^ 1) * T::M + h]);
-      // ---- online softmax; P(i) into TMEM once PV(i - 1) has finished
+      // ---- online softmax. Rescaling O needs PV(i - 1) finished; writing
+      // P buffer i & 1 needs PV(i - 2) finished (implied by PV(i - 1): the
+      // PV MMAs complete in issue order).
       const bool grow = bmax > m_used + 8.0f;
       const float m_new = grow ? bmax : m_used;
-      if (i > 0) {
-        if (!(ok = mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1))) break;
-        tc_fence_after();
-      }
       if (i > 0 && __any_sync(0xffffffffu, grow)) {
-        const float alpha = grow ? exp2f(m_used - m_new) : 1.0f;
+        ok = mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1);
+        tc_fence_after();
+        const float alpha = grow ? ex2_approx(m_used - m_new) : 1.0f;
 #pragma unroll 1
-        for (int c = half * (T::VH / 2); c < (half + 1) * (T::VH / 2); c += 16) {
+        for (int c = half * (T::VH / 2); c < (half + 1) * (T::VH / 2) && ok; c += 16) {
           uint32_t o[16];
           tmem_ld16(tmem_base + lane_addr + T::COL_O + c, o);
           tmem_wait_ld();
@@ -386,19 +421,23 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
         tmem_wait_st();
         l *= alpha;
         l_mma *= alpha;
+      } else if (i > 1) {
+        ok = mbar_wait(&pv_done[i & 1], ((i >> 1) & 1) ^ 1);
       }
       m_used = m_new;
       uint32_t pk[16];
-      float lsum = 0.f, lsum_mma = 0.f;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f}, lm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const float p0 = exp2f(z[2 * j] - m_used);
-        const float p1 = exp2f(z[2 * j + 1] - m_used);
+        const float p0 = ex2_approx(z[2 * j] - m_used);
+        const float p1 = ex2_approx(z[2 * j + 1] - m_used);
         const __nv_bfloat162 pb2 = __floats2bfloat162_rn(p0, p1);
-        lsum += p0 + p1;
-        lsum_mma += __low2float(pb2) + __high2float(pb2);
+        ls[j & 3] += p0 + p1;
+        lm[j & 3] += __low2float(pb2) + __high2float(pb2);
         pk[j] = *reinterpret_cast<const uint32_t*>(&pb2);
       }
+      float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+      float lsum_mma = (lm[0] + lm[1]) + (lm[2] + lm[3]);
       if (m_used == -INFINITY) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) pk[j] = 0u;
@@ -407,11 +446,15 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
       }
       l += lsum;
       l_mma += lsum_mma;
-      tmem_st16(tmem_base + lane_addr + col_s + half * 16, pk);
-      tmem_wait_st();
+      const uint32_t pb = p_row + (i & 1) * T::P_BYTES;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        sts_v4(pb + (((4 * half + c) ^ (h & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+               pk[4 * c + 3]);
+      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(p_full);
+      if (lane == 0) mbar_arrive(&p_full[i & 1]);
     }
     if (ok && n_blocks > 0) {
       ok = mbar_wait(&pv_done[(n_blocks - 1) & 1], ((n_blocks - 1) >> 1) & 1);
@@ -436,42 +479,66 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
     const float inv_l = has ? 1.0f / lm_all : 0.f;
     const uint32_t keep = has ? 0xffffffffu : 0u;   // masks undefined TMEM when empty
     const float lse_v = has ? (m_used + log2f(l_all)) * 0.69314718055994531f : -INFINITY;
+    // O leaves through the stage area (free now): each thread writes its
+    // row's 128 scaled columns there (16-byte chunk c of row h at chunk
+    // c ^ (h & 7)), then the eight softmax warps store whole rows, so every
+    // global store of a warp covers 512 contiguous bytes.
     const bool direct = p.splits == 1;
-    float* dst_f32 = nullptr;
-    __nv_bfloat16* dst_bf16 = nullptr;
-    if (direct) {
-      const size_t o_off = (static_cast<size_t>(row) * p.H + h) * T::DV + vh * T::VH;
-      if (p.out_bf16) dst_bf16 = static_cast<__nv_bfloat16*>(p.out) + o_off;
-      else dst_f32 = static_cast<float*>(p.out) + o_off;
-    } else {
-      const size_t part = static_cast<size_t>(row) * p.splits + split;
-      dst_f32 = p.part_o + (part * p.H + h) * T::DV + vh * T::VH;
-    }
+    const bool bf16_out = direct && p.out_bf16;
+    const int row_bytes = T::VH * (bf16_out ? 2 : 4);
+    const int n_chunks = row_bytes / 16;
+    uint8_t* o_stage = smem + T::OFF_OSTAGE;
+    {
+      const uint32_t row_base = smem_u32(o_stage) + h * row_bytes;
 #pragma unroll 1
-    for (int c = half * (T::VH / 2); c < (half + 1) * (T::VH / 2); c += 16) {
-      uint32_t o[16];
-      tmem_ld16(tmem_base + lane_addr + T::COL_O + c, o);
-      tmem_wait_ld();
+      for (int c = half * (T::VH / 2); c < (half + 1) * (T::VH / 2); c += 16) {
+        uint32_t o[16];
+        tmem_ld16(tmem_base + lane_addr + T::COL_O + c, o);
+        tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 16; ++j) o[j] &= keep;
-      if (h < p.H) {
-        if (dst_bf16) {
+        for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j] & keep) * inv_l);
+        if (bf16_out) {
           uint32_t pkd[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const __nv_bfloat162 v = __floats2bfloat162_rn(__uint_as_float(o[2 * j]) * inv_l,
-                                                           __uint_as_float(o[2 * j + 1]) * inv_l);
+            const __nv_bfloat162 v =
+                __floats2bfloat162_rn(__uint_as_float(o[2 * j]), __uint_as_float(o[2 * j + 1]));
             pkd[j] = *reinterpret_cast<const uint32_t*>(&v);
           }
-          reinterpret_cast<uint4*>(dst_bf16 + c)[0] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
-          reinterpret_cast<uint4*>(dst_bf16 + c)[1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
-        } else {
+          const int c0 = c / 8;                  // 16-byte chunk of column c (bf16)
 #pragma unroll
-          for (int j = 0; j < 16; j += 4)
-            reinterpret_cast<float4*>(dst_f32 + c)[j / 4] =
-                make_float4(__uint_as_float(o[j]) * inv_l, __uint_as_float(o[j + 1]) * inv_l,
-                            __uint_as_float(o[j + 2]) * inv_l, __uint_as_float(o[j + 3]) * inv_l);
+          for (int q = 0; q < 2; ++q)
+            sts_v4(row_base + (((c0 + q) ^ (h & 7)) << 4), pkd[4 * q], pkd[4 * q + 1],
+                   pkd[4 * q + 2], pkd[4 * q + 3]);
+        } else {
+          const int c0 = c / 4;                  // 16-byte chunk of column c (fp32)
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            sts_v4(row_base + (((c0 + q) ^ (h & 7)) << 4), o[4 * q], o[4 * q + 1], o[4 * q + 2],
+                   o[4 * q + 3]);
         }
+      }
+    }
+    named_bar_sync(5u, 32u * T::SOFTMAX_WARPS);
+    {
+      uint8_t* dst_base;
+      size_t dst_row_stride;                     // bytes between head rows
+      if (direct) {
+        const size_t o_off = (static_cast<size_t>(row) * p.H) * T::DV + vh * T::VH;
+        dst_base = bf16_out ? reinterpret_cast<uint8_t*>(static_cast<__nv_bfloat16*>(p.out) + o_off)
+                            : reinterpret_cast<uint8_t*>(static_cast<float*>(p.out) + o_off);
+      } else {
+        const size_t part = static_cast<size_t>(row) * p.splits + split;
+        dst_base = reinterpret_cast<uint8_t*>(p.part_o + (part * p.H) * T::DV + vh * T::VH);
+      }
+      dst_row_stride = static_cast<size_t>(T::DV) * (bf16_out ? 2 : 4);
+      const int tid = threadIdx.x - 5 * 32;      // 0..255 over the softmax warps
+      const int total = p.H * n_chunks;
+#pragma unroll 4
+      for (int k = tid; k < total; k += 32 * T::SOFTMAX_WARPS) {
+        const int r = k / n_chunks, ch = k - r * n_chunks;
+        const uint4 v = lds_v4(smem_u32(o_stage) + r * row_bytes + ((ch ^ (r & 7)) << 4));
+        *reinterpret_cast<uint4*>(dst_base + r * dst_row_stride + ch * 16) = v;
       }
     }
     if (vh == 0 && half == 0 && h < p.H) {

@@ -8,9 +8,9 @@
 //      radix passes over the samples find the 16-bit key prefix of the
 //      sample ranked about 1.25 k / n of the way down; tau is the lowest key
 //      with that prefix, so roughly 1.25 k keys of the row are >= tau.
-//   2. One pass over the row (16-byte loads, 16 scores per thread in flight)
+//   2. One pass over the row (16-byte loads, 32 scores per thread in flight)
 //      appends every (key, index) with key >= tau to a candidate buffer in
-//      shared memory (warp-aggregated slots).
+//      shared memory (one slot reservation per warp and round).
 //   3. If k <= #candidates <= capacity, an MSB-first radix select over the
 //      candidates finds the exact k-th key u*; every candidate above u* is
 //      written, then the lowest-index candidates equal to u*.
@@ -47,25 +47,34 @@ struct TopkSmem {
   uint32_t cand_u[kTopkCap];
   int32_t cand_i[kTopkCap];
   uint32_t samp[kTopkSamples];
-  uint32_t hist[256];
+  uint32_t hist[2][256];          // radix passes alternate buffers
   uint32_t warp_tot[kTopkThreads / 32];
-  uint32_t sel_bin, above, count, n_cand;
+  uint32_t sel_bin[2], above[2], sel_count[2];
+  uint32_t count, n_cand;
 };
 
 // Exact k-th largest key among `n` keys given by get(i) (all threads of the
 // CTA call this). Returns u*; *need_out = number of keys equal to u* that
 // belong to the top k; *eq_out = number of keys equal to u*.
-// With passes < 4 only the top 8 * passes bits are resolved: the result is
-// that prefix (low bits zero) of the k-th largest key.
-template <class Get>
+// With PASSES = 2 only the top 16 bits are resolved: the result is that
+// prefix (low bits zero) of the k-th largest key.
+// Pass p counts into hist[p & 1] while the other buffer is cleared for pass
+// p + 1, so a pass needs two CTA barriers. hist[0] is zero on entry and,
+// PASSES being even, is cleared again by the last pass before its barriers.
+template <int PASSES, class Get>
 __device__ uint32_t radix_kth(TopkSmem& sm, int n, uint32_t k, Get get, uint32_t* need_out,
-                              uint32_t* eq_out, int passes = 4) {
+                              uint32_t* eq_out) {
+  static_assert(PASSES == 2 || PASSES == 4, "an even number of 8-bit passes");
+  constexpr int passes = PASSES;
   const int tid = threadIdx.x;
   uint32_t prefix = 0, mask = 0, need = k, eq_count = 0;
   for (int pass = 0; pass < passes; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int i = tid; i < 256; i += kTopkThreads) sm.hist[i] = 0;
-    __syncthreads();
+    const int hb = pass & 1;
+    uint32_t* hist = sm.hist[hb];
+    // the other buffer: its last reader (the previous pass's scan) finished
+    // before that pass's second barrier
+    if (tid < 256) sm.hist[hb ^ 1][tid] = 0;
     for (int c0 = 0; c0 < n; c0 += kTopkThreads) {
       const int i = c0 + tid;
       uint32_t bin = 256u;
@@ -75,14 +84,14 @@ __device__ uint32_t radix_kth(TopkSmem& sm, int n, uint32_t k, Get get, uint32_t
       }
       // lanes with the same bin merge into one atomic (keys cluster in few bins)
       const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (bin < 256u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], __popc(peers));
+      if (bin < 256u && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
     }
     __syncthreads();
     if (tid < 32) {
       uint32_t c[8], sum = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        c[j] = sm.hist[255 - (tid * 8 + j)];
+        c[j] = hist[255 - (tid * 8 + j)];
         sum += c[j];
       }
       uint32_t incl = sum;
@@ -97,20 +106,19 @@ __device__ uint32_t radix_kth(TopkSmem& sm, int n, uint32_t k, Get get, uint32_t
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           if (acc < need && need <= acc + c[j]) {
-            sm.sel_bin = 255u - (tid * 8 + j);
-            sm.above = acc;
-            sm.count = c[j];
+            sm.sel_bin[hb] = 255u - (tid * 8 + j);
+            sm.above[hb] = acc;
+            sm.sel_count[hb] = c[j];
           }
           acc += c[j];
         }
       }
     }
     __syncthreads();
-    need -= sm.above;
-    eq_count = sm.count;
-    prefix |= sm.sel_bin << shift;
+    need -= sm.above[hb];
+    eq_count = sm.sel_count[hb];
+    prefix |= sm.sel_bin[hb] << shift;
     mask |= 255u << shift;
-    __syncthreads();
   }
   *need_out = need;
   *eq_out = eq_count;
@@ -138,29 +146,36 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
   // ---- 1. threshold: the 16-bit key prefix of the sample of rank `want`
   sm.samp[tid] = order_key(row[static_cast<int>((static_cast<int64_t>(tid) * n) / kTopkSamples)]);
   if (tid == 0) sm.n_cand = 0;
+  if (tid < 256) sm.hist[0][tid] = 0;
   __syncthreads();
   const int64_t want =
       (static_cast<int64_t>(5) * p.k * kTopkSamples) / (4 * static_cast<int64_t>(n)) + 8;
   uint32_t s_need, s_eq;
-  const uint32_t tau = radix_kth(
+  const uint32_t tau = radix_kth<2>(
       sm, kTopkSamples, static_cast<uint32_t>(want < kTopkSamples ? want : kTopkSamples),
-      [&](int i) { return sm.samp[i]; }, &s_need, &s_eq, 2);
+      [&](int i) { return sm.samp[i]; }, &s_need, &s_eq);
 
-  // ---- 2. one pass: candidates >= tau. Sixteen scores per thread and round
-  // are loaded before any is appended, as four 16-byte loads when the row is
-  // 16-byte aligned, so that the L2 / HBM latency of the row overlaps.
-  auto append = [&](uint32_t u, int i) {
-    const bool take = i < n && u >= tau;
-    const uint32_t bal = __ballot_sync(0xffffffffu, take);
-    if (bal) {
-      uint32_t base = 0;
-      if (lane == 0) base = atomicAdd(&sm.n_cand, static_cast<uint32_t>(__popc(bal)));
-      base = __shfl_sync(0xffffffffu, base, 0);
-      const uint32_t slot = base + __popc(bal & ((1u << lane) - 1u));
-      if (take && slot < static_cast<uint32_t>(kTopkCap)) {
-        sm.cand_u[slot] = u;
-        sm.cand_i[slot] = i;
-      }
+  // ---- 2. one pass: candidates >= tau. A thread takes 32 scores per round
+  // (eight 16-byte loads in flight when the row is 16-byte aligned) and
+  // forms a bit mask of those >= tau; the warp then reserves all of its
+  // slots with one shared atomic, each thread's first slot coming from an
+  // inclusive scan of the per-thread counts.
+  auto reserve = [&](uint32_t cnt) -> uint32_t {
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+    uint32_t base = 0;
+    if (lane == 0 && total) base = atomicAdd(&sm.n_cand, total);
+    return __shfl_sync(0xffffffffu, base, 0) + incl - cnt;
+  };
+  auto put = [&](uint32_t slot, uint32_t u, int i) {
+    if (slot < static_cast<uint32_t>(kTopkCap)) {
+      sm.cand_u[slot] = u;
+      sm.cand_i[slot] = i;
     }
   };
   int scalar_from = 0;   // scores [scalar_from, n) take the scalar loop
@@ -169,34 +184,48 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
     const float4* row4 = reinterpret_cast<const float4*>(row);
     const int n4 = n >> 2;
     scalar_from = n4 * 4;
-    for (int c0 = 0; c0 < n4; c0 += 4 * kTopkThreads) {
-      float4 v[4];
+    for (int c0 = 0; c0 < n4; c0 += 8 * kTopkThreads) {
+      uint4 v[8];                                  // order keys of 4 scores each
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
+      for (int m = 0; m < 8; ++m) {
         const int c = c0 + tid + m * kTopkThreads;
-        v[m] = c < n4 ? row4[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 f = c < n4 ? row4[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[m] = make_uint4(order_key(f.x), order_key(f.y), order_key(f.z), order_key(f.w));
       }
+      uint32_t mask = 0;
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        // past the last whole float4: an index >= n, so nothing is appended
-        const int c = c0 + tid + m * kTopkThreads;
-        const int i = c < n4 ? c * 4 : n;
-        append(order_key(v[m].x), i);
-        append(order_key(v[m].y), i + 1);
-        append(order_key(v[m].z), i + 2);
-        append(order_key(v[m].w), i + 3);
+      for (int m = 0; m < 8; ++m) {
+        // past the last whole float4 nothing is taken
+        const bool in = c0 + tid + m * kTopkThreads < n4;
+        mask |= static_cast<uint32_t>(in && v[m].x >= tau) << (4 * m);
+        mask |= static_cast<uint32_t>(in && v[m].y >= tau) << (4 * m + 1);
+        mask |= static_cast<uint32_t>(in && v[m].z >= tau) << (4 * m + 2);
+        mask |= static_cast<uint32_t>(in && v[m].w >= tau) << (4 * m + 3);
+      }
+      uint32_t slot = reserve(__popc(mask));
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int i = (c0 + tid + m * kTopkThreads) * 4;
+        if ((mask >> (4 * m)) & 1u) put(slot++, v[m].x, i);
+        if ((mask >> (4 * m + 1)) & 1u) put(slot++, v[m].y, i + 1);
+        if ((mask >> (4 * m + 2)) & 1u) put(slot++, v[m].z, i + 2);
+        if ((mask >> (4 * m + 3)) & 1u) put(slot++, v[m].w, i + 3);
       }
     }
   }
-  for (int c0 = scalar_from; c0 < n; c0 += 16 * kTopkThreads) {
-    uint32_t u[16];
+  for (int c0 = scalar_from; c0 < n; c0 += 32 * kTopkThreads) {
+    uint32_t u[32];
+    uint32_t mask = 0;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
+    for (int m = 0; m < 32; ++m) {
       const int i = c0 + tid + m * kTopkThreads;
       u[m] = i < n ? order_key(row[i]) : 0u;
+      mask |= static_cast<uint32_t>(i < n && u[m] >= tau) << m;
     }
+    uint32_t slot = reserve(__popc(mask));
 #pragma unroll
-    for (int m = 0; m < 16; ++m) append(u[m], c0 + tid + m * kTopkThreads);
+    for (int m = 0; m < 32; ++m)
+      if ((mask >> m) & 1u) put(slot++, u[m], c0 + tid + m * kTopkThreads);
   }
   __syncthreads();
   const uint32_t n_cand = sm.n_cand;
@@ -205,7 +234,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
   if (n_cand >= k && n_cand <= static_cast<uint32_t>(kTopkCap)) {
     // ---- 3. exact select among the candidates
     uint32_t need, eq_count;
-    const uint32_t kth = radix_kth(sm, static_cast<int>(n_cand), k,
+    const uint32_t kth = radix_kth<4>(sm, static_cast<int>(n_cand), k,
                                    [&](int i) { return sm.cand_u[i]; }, &need, &eq_count);
     if (tid == 0) sm.count = 0;
     __syncthreads();
@@ -239,7 +268,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
 
   // ---- fallback: exact select over the whole row (global memory per pass)
   uint32_t need, eq_count;
-  const uint32_t kth = radix_kth(sm, n, k, [&](int i) { return order_key(row[i]); }, &need,
+  const uint32_t kth = radix_kth<4>(sm, n, k, [&](int i) { return order_key(row[i]); }, &need,
                                  &eq_count);
   if (tid == 0) sm.count = 0;
   __syncthreads();
