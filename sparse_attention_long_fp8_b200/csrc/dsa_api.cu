@@ -391,7 +391,7 @@ dsa_status launch_topk(const dsa_shape* s, const HostLayout& lay, const float* s
   p.k = s->topk;
   p.out_rows = out_rows;
   p.out_row0 = out_row0;
-  dim3 grid(rows, s->batch);
+  dim3 grid(2 * rows, s->batch);   // a cluster of two CTAs per row
   dsa::topk_kernel<<<grid, dsa::kTopkThreads, smem, stream>>>(p);
   DSA_CUDA_TRY(cudaGetLastError(), "top-k launch");
   return DSA_OK;

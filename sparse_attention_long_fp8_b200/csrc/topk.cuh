@@ -2,15 +2,18 @@
 // 细粒度 Token 选择机制", eq. u_t: keep the k keys with the largest index
 // score). Ties are broken by the lower key index.
 //
-// One CTA per score row. Scores are mapped to order-preserving uint32 keys
-// (larger float <=> larger key; -0 is folded into +0).
+// A cluster of two CTAs per score row. Scores are mapped to order-preserving
+// uint32 keys (larger float <=> larger key; -0 is folded into +0).
 //   1. A threshold tau from 1024 evenly spaced samples of the row: two 8-bit
 //      radix passes over the samples find the 16-bit key prefix of the
 //      sample ranked about 1.25 k / n of the way down; tau is the lowest key
 //      with that prefix, so roughly 1.25 k keys of the row are >= tau.
-//   2. One pass over the row (16-byte loads, 32 scores per thread in flight)
-//      appends every (key, index) with key >= tau to a candidate buffer in
-//      shared memory (one slot reservation per warp and round).
+//   2. Each CTA of the pair takes one half of the row (16-byte loads, 32
+//      scores per thread in flight) and appends every (key, index) with key
+//      >= tau to its own candidate buffer in shared memory (one slot
+//      reservation per warp and round). Both compute the same tau from the
+//      same samples. CTA 1's candidates are then read by CTA 0 over
+//      distributed shared memory; CTA 0 alone does the rest.
 //   3. If k <= #candidates <= capacity, an MSB-first radix select over the
 //      candidates finds the exact k-th key u*; every candidate above u* is
 //      written, then the lowest-index candidates equal to u*.
@@ -125,11 +128,13 @@ __device__ uint32_t radix_kth(TopkSmem& sm, int n, uint32_t k, Get get, uint32_t
   return prefix;
 }
 
-__global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTopkThreads, 1)
+    topk_kernel(TopkParams p) {
   extern __shared__ __align__(16) uint8_t tk_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_raw);
 
-  const int r = blockIdx.x, b = blockIdx.y;
+  const int r = blockIdx.x >> 1, b = blockIdx.y;
+  const uint32_t part = cluster_ctarank();     // which half of the row this CTA scans
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int pos = p.rp.pos(b, p.row_begin + r);
   const int kvl = min(p.kv_len ? p.kv_len[b] : p.n_kv, p.n_kv);
@@ -138,8 +143,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
   int32_t* out = p.indices + (static_cast<size_t>(b) * p.out_rows + p.out_row0 + r) * p.k;
   const uint32_t k = static_cast<uint32_t>(p.k);
 
-  if (n <= p.k) {
-    for (int i = tid; i < p.k; i += kTopkThreads) out[i] = i < n ? i : -1;
+  if (n <= p.k) {   // both CTAs of the pair leave here (same row, same n)
+    if (part == 0)
+      for (int i = tid; i < p.k; i += kTopkThreads) out[i] = i < n ? i : -1;
     return;
   }
 
@@ -178,25 +184,29 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
       sm.cand_i[slot] = i;
     }
   };
-  int scalar_from = 0;   // scores [scalar_from, n) take the scalar loop
+  // this CTA's scores: [lo, hi) as whole float4s when the row is 16-byte
+  // aligned (the < 4 scores past the last whole float4 go to CTA 1's scalar
+  // loop), else [s_lo, s_hi) by the scalar loop alone
+  int s_lo, s_hi;
   if ((reinterpret_cast<uintptr_t>(row) & 15u) == 0) {
-    // whole float4s inside [0, n) only; the tail (< 4 scores) below
     const float4* row4 = reinterpret_cast<const float4*>(row);
-    const int n4 = n >> 2;
-    scalar_from = n4 * 4;
-    for (int c0 = 0; c0 < n4; c0 += 8 * kTopkThreads) {
+    const int n4 = n >> 2, h4 = (n4 + 1) >> 1;
+    const int lo4 = part ? h4 : 0, hi4 = part ? n4 : h4;
+    s_lo = part ? n4 * 4 : n;
+    s_hi = n;
+    for (int c0 = lo4; c0 < hi4; c0 += 8 * kTopkThreads) {
       uint4 v[8];                                  // order keys of 4 scores each
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
         const int c = c0 + tid + m * kTopkThreads;
-        const float4 f = c < n4 ? row4[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 f = c < hi4 ? row4[c] : make_float4(0.f, 0.f, 0.f, 0.f);
         v[m] = make_uint4(order_key(f.x), order_key(f.y), order_key(f.z), order_key(f.w));
       }
       uint32_t mask = 0;
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
-        // past the last whole float4 nothing is taken
-        const bool in = c0 + tid + m * kTopkThreads < n4;
+        // past this CTA's last float4 nothing is taken
+        const bool in = c0 + tid + m * kTopkThreads < hi4;
         mask |= static_cast<uint32_t>(in && v[m].x >= tau) << (4 * m);
         mask |= static_cast<uint32_t>(in && v[m].y >= tau) << (4 * m + 1);
         mask |= static_cast<uint32_t>(in && v[m].z >= tau) << (4 * m + 2);
@@ -212,26 +222,47 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(TopkParams p) {
         if ((mask >> (4 * m + 3)) & 1u) put(slot++, v[m].w, i + 3);
       }
     }
+  } else {
+    const int half_n = (n + 1) >> 1;
+    s_lo = part ? half_n : 0;
+    s_hi = part ? n : half_n;
   }
-  for (int c0 = scalar_from; c0 < n; c0 += 32 * kTopkThreads) {
+  for (int c0 = s_lo; c0 < s_hi; c0 += 32 * kTopkThreads) {
     uint32_t u[32];
     uint32_t mask = 0;
 #pragma unroll
     for (int m = 0; m < 32; ++m) {
       const int i = c0 + tid + m * kTopkThreads;
-      u[m] = i < n ? order_key(row[i]) : 0u;
-      mask |= static_cast<uint32_t>(i < n && u[m] >= tau) << m;
+      u[m] = i < s_hi ? order_key(row[i]) : 0u;
+      mask |= static_cast<uint32_t>(i < s_hi && u[m] >= tau) << m;
     }
     uint32_t slot = reserve(__popc(mask));
 #pragma unroll
     for (int m = 0; m < 32; ++m)
       if ((mask >> m) & 1u) put(slot++, u[m], c0 + tid + m * kTopkThreads);
   }
-  __syncthreads();
-  const uint32_t n_cand = sm.n_cand;
-  __syncthreads();
+  // ---- CTA 0 takes CTA 1's candidates behind its own
+  cluster_sync();                  // both candidate buffers and counts are final
+  if (part != 0) {
+    cluster_sync();                // CTA 0 has read this CTA's shared memory
+    return;
+  }
+  const uint32_t n_own = sm.n_cand;
+  const uint32_t n_peer = ld_dsmem_u32(mapa_shared(smem_u32(&sm.n_cand), 1));
+  const uint32_t cap = static_cast<uint32_t>(kTopkCap);
+  const bool fits = n_own <= cap && n_peer <= cap && n_own + n_peer <= cap;
+  if (fits) {
+    const uint32_t pu = mapa_shared(smem_u32(&sm.cand_u[0]), 1);
+    const uint32_t pi = mapa_shared(smem_u32(&sm.cand_i[0]), 1);
+    for (uint32_t j = tid; j < n_peer; j += kTopkThreads) {
+      sm.cand_u[n_own + j] = ld_dsmem_u32(pu + 4 * j);
+      sm.cand_i[n_own + j] = static_cast<int32_t>(ld_dsmem_u32(pi + 4 * j));
+    }
+  }
+  cluster_sync();
+  const uint32_t n_cand = fits ? n_own + n_peer : cap + 1;
 
-  if (n_cand >= k && n_cand <= static_cast<uint32_t>(kTopkCap)) {
+  if (n_cand >= k && n_cand <= cap) {
     // ---- 3. exact select among the candidates
     uint32_t need, eq_count;
     const uint32_t kth = radix_kth<4>(sm, static_cast<int>(n_cand), k,
