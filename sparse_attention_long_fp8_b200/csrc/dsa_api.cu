@@ -505,10 +505,13 @@ dsa_status launch_attn_vh(const dsa_shape* s, const dsa::KeyMap& km, const AttnP
     p.part_o = static_cast<float*>(ws);
     p.part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + (po + 255) / 256 * 256);
   }
-  const int64_t nblocks = rows * pl.splits * 2;
-  if (nblocks >= (1ll << 31)) return fail(DSA_ERR_INVALID_ARG, "too many attention rows");
-  dsa::sparse_attn_vh_kernel<<<static_cast<unsigned>(nblocks), T::THREADS, T::SMEM_BYTES, stream>>>(
-      p);
+  // persistent CTAs (one per SM, an even number so that a CTA keeps its
+  // value half), each walking units c, c + grid, ...
+  const int64_t n_units = rows * pl.splits * 2;
+  if (n_units >= (1ll << 31)) return fail(DSA_ERR_INVALID_ARG, "too many attention rows");
+  const int64_t grid = std::min<int64_t>(n_units, std::max(2, num_sms() / 2 * 2));
+  dsa::sparse_attn_vh_kernel<<<static_cast<unsigned>(grid), T::THREADS, T::SMEM_BYTES, stream>>>(
+      p, n_units);
   DSA_CUDA_TRY(cudaGetLastError(), "sparse attention launch");
   if (pl.splits > 1) {
     dim3 grid(static_cast<unsigned>(rows), s->heads);

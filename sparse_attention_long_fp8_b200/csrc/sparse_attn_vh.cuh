@@ -31,6 +31,12 @@
 // TMEM per CTA: O 256 columns, S 64, Q 192 (six 64-dim blocks: the five that
 // only the logits read and the first of the V half) = 512. Q's other three
 // V-half blocks are in shared memory.
+//
+// The CTAs are persistent: CTA c takes units c, c + grid, ... (a unit is one
+// (query row, split, value half)), and every barrier phase runs on across
+// units. At the end of a unit the softmax warps load the next unit's Q (its
+// S MMAs can then start) before they write this unit's O, and the next
+// unit's Q row is prefetched into L2 while the current unit runs.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -65,10 +71,8 @@ struct VhTile {
   static constexpr int OFF_QS = STAGES * STAGE_BYTES;
   static constexpr int OFF_P = OFF_QS + QS_BYTES;            // [2] P tiles
   static constexpr int OFF_RED = OFF_P + 2 * P_BYTES;        // [2 parity][2 halves][128] fp32
-  static constexpr int OFF_END = OFF_C;      // [half][l, l_mma][128] fp32, after the last PV
-  static constexpr int OFF_OSTAGE = OFF_C + 4096;            // O rows on their way out
   static constexpr int OFF_BAR = OFF_RED + 2 * 2 * M * 4;
-  static constexpr int NUM_BARS = 4 * STAGES + 7 + 4;        // stages, singles, end[4]
+  static constexpr int NUM_BARS = 4 * STAGES + 7;            // stages, then the singles
   // No alignment slack: the dynamic shared memory of this kernel starts on a
   // 1024-byte boundary (checked at run time; a misaligned base is reported).
   static constexpr int SMEM_BYTES = OFF_BAR + NUM_BARS * 8 + 16;
@@ -76,7 +80,6 @@ struct VhTile {
   static_assert(STAGE_BYTES % 1024 == 0 && OFF_QS % 1024 == 0 && OFF_P % 1024 == 0,
                 "1024-byte aligned operands");
   static_assert(COL_S + NK == COL_Q && COL_Q + XT * 32 == 512, "TMEM columns");
-  static_assert(OFF_OSTAGE + M * VH * 4 <= OFF_QS, "O staging fits in the stage area");
 };
 
 // Latent dim block of the t-th Q block held in TMEM (t = 0..5): the other
@@ -88,11 +91,30 @@ __device__ __forceinline__ int vh_tblock(int t, int v) {
 }
 __device__ __forceinline__ int vh_sblock(int u, int v) { return 4 * v + 1 + u; }
 
+// Unit u of 2 * rows * splits: value half u & 1 of (row, split) = u >> 1.
+struct VhUnit {
+  int vh, row, split, b, slot_begin, slot_end, n_blocks;
+  const int32_t* row_idx;
+};
+__device__ __forceinline__ VhUnit vh_unit(const AttnParams& p, int64_t u) {
+  VhUnit w;
+  w.vh = static_cast<int>(u & 1);
+  const int64_t pair = u >> 1;
+  w.row = static_cast<int>(pair / p.splits);
+  w.split = static_cast<int>(pair % p.splits);
+  w.b = w.row / p.n_q;
+  w.slot_begin = w.split * p.slots_per_split;
+  w.slot_end = min(p.topk, w.slot_begin + p.slots_per_split);
+  w.n_blocks = max(0, (w.slot_end - w.slot_begin + VhTile::NK - 1) / VhTile::NK);
+  w.row_idx = p.indices + static_cast<size_t>(w.row) * p.topk;
+  return w;
+}
+
 // Warp roles: 0-3 gather (cp.async, 16 bytes per copy); 4 issues
 // the logit MMAs and owns TMEM; 5-12 run the softmax (two warps per TMEM lane
 // quarter: a thread owns one head row and 32 of a block's 64 keys); 13 issues
 // the PV MMAs.
-__global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
+__global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, int64_t n_units) {
   using T = VhTile;
   constexpr int NK = T::NK;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -108,8 +130,7 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
   uint64_t* s_free = s_full + 1;                 // S tile loaded by all softmax warps
   uint64_t* p_full = s_full + 2;                 // [2] P tile of buffer b written
   uint64_t* pv_done = s_full + 4;                // [2] PV of buffer b finished (buffer free, O updated)
-  uint64_t* q_ready = s_full + 6;                // Q in TMEM and shared memory
-  uint64_t* end_bar = s_full + 7;                // [quarter]: both halves of l, l_mma written
+  uint64_t* q_ready = s_full + 6;                // Q of a unit in TMEM and shared memory
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + T::NUM_BARS);
 
   if ((smem_u32(smem_raw) & 1023u) != 0) {      // see SMEM_BYTES: no slack to realign
@@ -118,15 +139,7 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
   }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int vh = blockIdx.x & 1;                 // value half of this CTA
-  const int unit = blockIdx.x >> 1;
-  const int row = unit / p.splits;               // b * n_q + t
-  const int split = unit % p.splits;
-  const int b = row / p.n_q;
-  const int slot_begin = split * p.slots_per_split;
-  const int slot_end = min(p.topk, slot_begin + p.slots_per_split);
-  const int n_blocks = max(0, (slot_end - slot_begin + NK - 1) / NK);
-  const int32_t* row_idx = p.indices + static_cast<size_t>(row) * p.topk;
+  const int64_t u0 = blockIdx.x, du = gridDim.x;   // this CTA's units: u0, u0 + du, ...
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < T::STAGES; ++s) {
@@ -142,7 +155,6 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
       mbar_init(&pv_done[s], 1);
     }
     mbar_init(q_ready, T::SOFTMAX_WARPS);
-    for (int s = 0; s < 4; ++s) mbar_init(&end_bar[s], 2);
     fence_mbar_init();
   }
   if (warp == 4) {
@@ -154,6 +166,10 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Every role walks the same units and counts their blocks alike: g is the
+  // CTA's running block number, which picks the stage, the P buffer and the
+  // barrier phases. Units with no blocks (a split past the top-k slots) only
+  // get their empty output.
   if (warp < 4) {
     // ------------------------------------------------------------ gather
     // Thread (kq = tid / 8, ch = tid % 8) copies 16-byte chunk ch of every
@@ -165,14 +181,6 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
     // instruction moves four whole 128-byte lines.
     const int kq = threadIdx.x >> 3, ch = threadIdx.x & 7;
     const uint32_t dst0 = smem_u32(c_smem) + kq * 128 + ((ch ^ (kq & 7)) << 4);
-    auto load_keys = [&](int blk, int64_t (&k)[4]) {
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int slot = slot_begin + blk * NK + kq + 16 * r;
-        const int idx = (blk < n_blocks && slot < slot_end) ? row_idx[slot] : -1;
-        k[r] = (idx >= 0 && idx < p.n_kv) ? p.km.row(b, idx, p.n_kv) : -1;   // pool row
-      }
-    };
     auto copy_part = [&](auto vh_c, auto vpart_c, uint32_t dst, const __nv_bfloat16* const (&src)[4],
                          const uint32_t (&bytes)[4]) {
       constexpr int V = decltype(vh_c)::value;
@@ -189,31 +197,43 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
     using I1 = std::integral_constant<int, 1>;
     using BX = std::integral_constant<bool, false>;
     using BV = std::integral_constant<bool, true>;
-    int64_t keys[4];
-    load_keys(0, keys);
+    uint32_t g = 0;
     bool ok = true;
-    for (int i = 0; i < n_blocks && ok; ++i) {
-      const int st = i % T::STAGES;
-      const uint32_t ph = ((i / T::STAGES) & 1) ^ 1;
-      const __nv_bfloat16* src[4];
-      uint32_t bytes[4];
+    for (int64_t u = u0; u < n_units && ok; u += du) {
+      const VhUnit w = vh_unit(p, u);
+      auto load_keys = [&](int blk, int64_t (&k)[4]) {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        src[r] = p.kv + (keys[r] >= 0 ? keys[r] : 0) * T::DQK + ch * 8;
-        bytes[r] = keys[r] >= 0 ? 16u : 0u;
+        for (int r = 0; r < 4; ++r) {
+          const int slot = w.slot_begin + blk * NK + kq + 16 * r;
+          const int idx = (blk < w.n_blocks && slot < w.slot_end) ? w.row_idx[slot] : -1;
+          k[r] = (idx >= 0 && idx < p.n_kv) ? p.km.row(w.b, idx, p.n_kv) : -1;   // pool row
+        }
+      };
+      int64_t keys[4];
+      load_keys(0, keys);
+      for (int i = 0; i < w.n_blocks && ok; ++i, ++g) {
+        const int st = g % T::STAGES;
+        const uint32_t ph = ((g / T::STAGES) & 1) ^ 1;
+        const __nv_bfloat16* src[4];
+        uint32_t bytes[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          src[r] = p.kv + (keys[r] >= 0 ? keys[r] : 0) * T::DQK + ch * 8;
+          bytes[r] = keys[r] >= 0 ? 16u : 0u;
+        }
+        load_keys(i + 1, keys);   // one block ahead
+        const uint32_t dst = dst0 + st * T::STAGE_BYTES;
+        ok = mbar_wait(&cx_empty[st], ph);
+        if (!ok) break;
+        if (w.vh == 0) copy_part(I0{}, BX{}, dst, src, bytes);
+        else copy_part(I1{}, BX{}, dst, src, bytes);
+        cp_async_arrive_noinc(&cx_full[st]);
+        ok = mbar_wait(&cv_empty[st], ph);
+        if (!ok) break;
+        if (w.vh == 0) copy_part(I0{}, BV{}, dst, src, bytes);
+        else copy_part(I1{}, BV{}, dst, src, bytes);
+        cp_async_arrive_noinc(&cv_full[st]);
       }
-      load_keys(i + 1, keys);   // one block ahead
-      const uint32_t dst = dst0 + st * T::STAGE_BYTES;
-      ok = mbar_wait(&cx_empty[st], ph);
-      if (!ok) break;
-      if (vh == 0) copy_part(I0{}, BX{}, dst, src, bytes);
-      else copy_part(I1{}, BX{}, dst, src, bytes);
-      cp_async_arrive_noinc(&cx_full[st]);
-      ok = mbar_wait(&cv_empty[st], ph);
-      if (!ok) break;
-      if (vh == 0) copy_part(I0{}, BV{}, dst, src, bytes);
-      else copy_part(I1{}, BV{}, dst, src, bytes);
-      cp_async_arrive_noinc(&cv_full[st]);
     }
     cp_async_wait_all();
   } else if (warp == 4) {
@@ -228,77 +248,91 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
       constexpr uint32_t idesc_s = umma_idesc(128, NK, 1u, 1u, 0u, 0u);
       const uint64_t c_desc0 = umma_desc(smem_u32(c_smem), 16, 1024, 2);
       const uint64_t q_desc0 = umma_desc(smem_u32(qs_smem), 16, 1024, 2);
-      const uint32_t x_shift = static_cast<uint32_t>(4 * (1 - vh) * T::DB_BYTES) >> 4;
-      const uint32_t v_shift = static_cast<uint32_t>(4 * vh * T::DB_BYTES) >> 4;
       const uint32_t d_s = tmem_base + T::COL_S;
-      bool ok = mbar_wait(q_ready, 0);
-      tc_fence_after();
-      for (int i = 0; i < n_blocks && ok; ++i) {
-        const int st = i % T::STAGES;
-        const uint32_t ph = (i / T::STAGES) & 1;
-        // the S buffer is free once every softmax warp has loaded S(i - 1)
-        ok = (i == 0 || mbar_wait(s_free, (i - 1) & 1)) && mbar_wait(&cx_full[st], ph);
-        if (!ok) break;
-        fence_proxy_async_smem();
+      uint32_t g = 0, k = 0;
+      bool ok = true;
+      for (int64_t u = u0; u < n_units && ok; u += du) {
+        const VhUnit w = vh_unit(p, u);
+        if (w.n_blocks == 0) continue;
+        const uint32_t x_shift = static_cast<uint32_t>(4 * (1 - w.vh) * T::DB_BYTES) >> 4;
+        const uint32_t v_shift = static_cast<uint32_t>(4 * w.vh * T::DB_BYTES) >> 4;
+        ok = mbar_wait(q_ready, k & 1);
+        ++k;
         tc_fence_after();
-        const uint64_t cd = c_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
-        // logit-only part of the stage (the other half's value blocks, then
-        // the RoPE block), Q from TMEM
+        for (int i = 0; i < w.n_blocks && ok; ++i, ++g) {
+          const int st = g % T::STAGES;
+          const uint32_t ph = (g / T::STAGES) & 1;
+          // the S buffer is free once every softmax warp has loaded S(g - 1)
+          ok = (g == 0 || mbar_wait(s_free, (g - 1) & 1)) && mbar_wait(&cx_full[st], ph);
+          if (!ok) break;
+          fence_proxy_async_smem();
+          tc_fence_after();
+          const uint64_t cd = c_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
+          // logit-only part of the stage (the other half's value blocks, then
+          // the RoPE block), Q from TMEM
 #pragma unroll
-        for (int t = 0; t < T::XDB; ++t)
+          for (int t = 0; t < T::XDB; ++t)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t off = (t < 4 ? t * T::DB_BYTES : 8 * T::DB_BYTES) + kk * 32;
+              const uint64_t bd = cd + (t < 4 ? x_shift : 0u) + (off >> 4);
+              umma_bf16_ts(d_s, tmem_base + T::COL_Q + t * 32 + kk * 8, bd, idesc_s,
+                           (t | kk) ? 1u : 0u);
+            }
+          umma_commit(&cx_empty[st]);
+          ok = mbar_wait(&cv_full[st], ph);
+          if (!ok) break;
+          fence_proxy_async_smem();
+          tc_fence_after();
+          // V-half blocks: the first with Q from TMEM, the other three from
+          // shared memory
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t off = (t < 4 ? t * T::DB_BYTES : 8 * T::DB_BYTES) + kk * 32;
-            const uint64_t bd = cd + (t < 4 ? x_shift : 0u) + (off >> 4);
-            umma_bf16_ts(d_s, tmem_base + T::COL_Q + t * 32 + kk * 8, bd, idesc_s,
-                         (t | kk) ? 1u : 0u);
+            const uint64_t bd = cd + v_shift + ((kk * 32) >> 4);
+            umma_bf16_ts(d_s, tmem_base + T::COL_Q + T::XDB * 32 + kk * 8, bd, idesc_s, 1u);
           }
-        umma_commit(&cx_empty[st]);
-        ok = mbar_wait(&cv_full[st], ph);
-        if (!ok) break;
-        fence_proxy_async_smem();
-        tc_fence_after();
-        // V-half blocks: the first with Q from TMEM, the other three from
-        // shared memory
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = cd + v_shift + ((kk * 32) >> 4);
-          umma_bf16_ts(d_s, tmem_base + T::COL_Q + T::XDB * 32 + kk * 8, bd, idesc_s, 1u);
+          for (int uq = 0; uq < T::QSB; ++uq)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = q_desc0 + ((uq * T::M * 128 + kk * 32) >> 4);
+              const uint64_t bd = cd + v_shift + (((uq + 1) * T::DB_BYTES + kk * 32) >> 4);
+              umma_bf16_ss(d_s, ad, bd, idesc_s, 1u);
+            }
+          umma_commit(s_full);
         }
-#pragma unroll
-        for (int u = 0; u < T::QSB; ++u)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = q_desc0 + ((u * T::M * 128 + kk * 32) >> 4);
-            const uint64_t bd = cd + v_shift + (((u + 1) * T::DB_BYTES + kk * 32) >> 4);
-            umma_bf16_ss(d_s, ad, bd, idesc_s, 1u);
-          }
-        umma_commit(s_full);
       }
     }
     __syncwarp();
   } else if (warp == 13) {
     // ------------------------------------------------------------ O += P V issuer
-    // P(j) exists only after S(j) was read, so S(j) has completed: when PV(j)
+    // P(g) exists only after S(g) was read, so S(g) has completed: when PV(g)
     // completes, both readers of the V-half blocks are done, and P buffer
-    // j & 1 is free. One elected lane issues (as for S).
+    // g & 1 is free. The first PV of a unit overwrites O: the softmax warps
+    // write that unit's first P only after they have read out the previous
+    // unit's O. One elected lane issues (as for S).
     if (elect_one()) {
       constexpr uint32_t idesc_pv = umma_idesc(128, T::VH, 1u, 1u, 0u, 1u);
-      const uint64_t v_desc0 =
-          umma_desc(smem_u32(c_smem) + 4 * vh * T::DB_BYTES, T::DB_BYTES, 1024, 2);
       const uint64_t p_desc0 = umma_desc(smem_u32(smem + T::OFF_P), 16, 1024, 2);
-      for (int j = 0; j < n_blocks; ++j) {
-        const int st = j % T::STAGES;
-        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1)) break;
-        tc_fence_after();
-        const uint64_t vd = v_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
-        const uint64_t pd = p_desc0 + static_cast<uint32_t>((j & 1) * (T::P_BYTES >> 4));
+      uint32_t g = 0;
+      bool ok = true;
+      for (int64_t u = u0; u < n_units && ok; u += du) {
+        const VhUnit w = vh_unit(p, u);
+        const uint64_t v_desc0 =
+            umma_desc(smem_u32(c_smem) + 4 * w.vh * T::DB_BYTES, T::DB_BYTES, 1024, 2);
+        for (int i = 0; i < w.n_blocks; ++i, ++g) {
+          const int st = g % T::STAGES;
+          if (!(ok = mbar_wait(&p_full[g & 1], (g >> 1) & 1))) break;
+          tc_fence_after();
+          const uint64_t vd = v_desc0 + static_cast<uint32_t>(st * (T::STAGE_BYTES >> 4));
+          const uint64_t pd = p_desc0 + static_cast<uint32_t>((g & 1) * (T::P_BYTES >> 4));
 #pragma unroll
-        for (int kk = 0; kk < NK / 16; ++kk)
-          umma_bf16_ss(tmem_base + T::COL_O, pd + ((kk * 32) >> 4), vd + ((kk * 2048) >> 4),
-                       idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(&cv_empty[st]);
-        umma_commit(&pv_done[j & 1]);
+          for (int kk = 0; kk < NK / 16; ++kk)
+            umma_bf16_ss(tmem_base + T::COL_O, pd + ((kk * 32) >> 4), vd + ((kk * 2048) >> 4),
+                         idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&cv_empty[st]);
+          umma_commit(&pv_done[g & 1]);
+        }
       }
     }
     __syncwarp();
@@ -308,245 +342,317 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p) {
     const int half = (warp - 5) >> 2;                        // which 32 keys of a block
     const int h = quarter * 32 + lane;                       // head row = TMEM lane
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t pair_bar = 1u + static_cast<uint32_t>(quarter);   // the quarter's two warps
     float* red = reinterpret_cast<float*>(smem + T::OFF_RED);   // [parity][half][128]
 
-    // Q into TMEM (six blocks; the two warps of a quarter take alternate
-    // 16-column chunks) and shared memory (three V-half blocks, K-major
-    // 128-byte swizzle; the two warps alternate blocks). The shared-memory
-    // part goes by cp.async, and every load of the TMEM part is issued before
-    // the first TMEM store, so the whole of Q costs one memory round trip.
-    {
-      const __nv_bfloat16* qh = p.q + (static_cast<size_t>(row) * p.H + min(h, p.H - 1)) * T::DQK;
-      const bool live = h < p.H;
+    const int stid = threadIdx.x - 5 * 32;                   // 0..255 over the softmax warps
+    constexpr uint32_t kAllBar = 5u;                         // named barrier of the 8 warps
+    constexpr uint32_t kAllThreads = 32u * T::SOFTMAX_WARPS;
+    // Q of a unit: rows of 1152 bytes, one per head. The 256 softmax threads
+    // copy three 64-dim blocks at a time into the Q area of shared memory
+    // (cp.async, 4 whole 128-byte lines per warp instruction, the K-major
+    // 128-byte-swizzled layout of the MMA operand): twice as staging for the
+    // six TMEM blocks, which every thread then moves from its own head row
+    // into its TMEM lane, and once more for the three blocks that stay there.
+    auto copy_q3 = [&](const VhUnit& w, int first, bool tmem_part) {
+      const __nv_bfloat16* qrow = p.q + static_cast<size_t>(w.row) * p.H * T::DQK;
+      const int r4 = stid >> 3, ch = stid & 7;
 #pragma unroll
-      for (int u = half; u < T::QSB; u += 2) {
-        const __nv_bfloat16* src = qh + vh_sblock(u, vh) * 64;
-        const uint32_t dst = smem_u32(qs_smem) + u * (T::M * 128) + (h >> 3) * 1024 + (h & 7) * 128;
+      for (int j = 0; j < 3; ++j) {
+        const int db = tmem_part ? vh_tblock(first + j, w.vh) : vh_sblock(first + j, w.vh);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          cp_async_16(dst + ((ch ^ (h & 7)) << 4), src + ch * 8, live ? 16u : 0u);
-      }
-      constexpr int NCH = T::XT;                 // TMEM chunks per warp (of 2 * XT)
-      uint4 qv[NCH][4];
-#pragma unroll
-      for (int k = 0; k < NCH; ++k) {
-        const int c = half + 2 * k;
-        const uint4* src =
-            reinterpret_cast<const uint4*>(qh + vh_tblock(c >> 1, vh) * 64 + (c & 1) * 32);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) qv[k][j] = live ? __ldg(src + j) : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll
-      for (int k = 0; k < NCH; ++k) {
-        uint32_t v[16];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          v[4 * j] = qv[k][j].x; v[4 * j + 1] = qv[k][j].y;
-          v[4 * j + 2] = qv[k][j].z; v[4 * j + 3] = qv[k][j].w;
+        for (int it = 0; it < T::M / 32; ++it) {
+          const int r = it * 32 + r4;
+          const __nv_bfloat16* src = qrow + static_cast<size_t>(min(r, p.H - 1)) * T::DQK + db * 64 + ch * 8;
+          const uint32_t dst = smem_u32(qs_smem) + j * (T::M * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
+                               ((ch ^ (r & 7)) << 4);
+          cp_async_16(dst, src, r < p.H ? 16u : 0u);
         }
-        tmem_st16(tmem_base + lane_addr + T::COL_Q + (half + 2 * k) * 16, v);
       }
       cp_async_wait_all();
+    };
+    auto load_q = [&](const VhUnit& w) {
+#pragma unroll 1
+      for (int round = 0; round < 2; ++round) {
+        copy_q3(w, 3 * round, true);
+        named_bar_sync(kAllBar, kAllThreads);
+        // this warp's 16-column chunk (32 dims: 16-byte chunks 4 half .. +3)
+        // of each staged block, from its lane's head row
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          const uint32_t rowp = smem_u32(qs_smem) + j * (T::M * 128) + (h >> 3) * 1024 + (h & 7) * 128;
+          uint32_t v[16];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 x = lds_v4(rowp + (((4 * half + c) ^ (h & 7)) << 4));
+            v[4 * c] = x.x; v[4 * c + 1] = x.y; v[4 * c + 2] = x.z; v[4 * c + 3] = x.w;
+          }
+          tmem_st16(tmem_base + lane_addr + T::COL_Q + (2 * (3 * round + j) + half) * 16, v);
+        }
+        named_bar_sync(kAllBar, kAllThreads);      // staging read before it is overwritten
+      }
+      copy_q3(w, 0, false);
       fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
-    }
-
-    float m_used = -INFINITY;   // running max (log2 domain) the P values are relative to
-    float l = 0.f;              // this warp's share of the sum of the fp32 p (LSE)
-    float l_mma = 0.f;          // ... of the bf16-rounded p the PV MMA used (normalises O)
-    bool ok = true;
-    auto load_idx = [&](int blk) -> int {
-      const int slot = slot_begin + blk * NK + half * 32 + lane;
-      return (blk < n_blocks && slot < slot_end) ? row_idx[slot] : -1;
     };
-    int idx_next = load_idx(0);
+    // The next unit's Q rows into L2 (a hint): 256 threads, one line each
+    // per step.
+    auto prefetch_unit = [&](int64_t u) {
+      if (u >= n_units) return;
+      const VhUnit w = vh_unit(p, u);
+      const char* q = reinterpret_cast<const char*>(p.q + static_cast<size_t>(w.row) * p.H * T::DQK);
+      const int lines = p.H * T::DQK * 2 / 128;
+      for (int l = stid; l < lines; l += kAllThreads) prefetch_l2(q + static_cast<size_t>(l) * 128);
+    };
+    // A unit without blocks (a split past the top-k slots): O = 0, LSE = -inf.
+    auto write_empty = [&](const VhUnit& w) {
+      if (h >= p.H) return;
+      const bool direct = p.splits == 1;
+      for (int c = half * (T::VH / 2); c < (half + 1) * (T::VH / 2); ++c) {
+        if (direct) {
+          const size_t o_off = (static_cast<size_t>(w.row) * p.H + h) * T::DV + w.vh * T::VH + c;
+          if (p.out_bf16) static_cast<__nv_bfloat16*>(p.out)[o_off] = __float2bfloat16(0.f);
+          else static_cast<float*>(p.out)[o_off] = 0.f;
+        } else {
+          const size_t part = static_cast<size_t>(w.row) * p.splits + w.split;
+          p.part_o[(part * p.H + h) * T::DV + w.vh * T::VH + c] = 0.f;
+        }
+      }
+      if (w.vh == 0 && half == 0) {
+        if (direct) {
+          if (p.lse) p.lse[static_cast<size_t>(w.row) * p.H + h] = -INFINITY;
+        } else {
+          p.part_lse[(static_cast<size_t>(w.row) * p.splits + w.split) * p.H + h] = -INFINITY;
+        }
+      }
+    };
+
     uint32_t sr[32];
     float z[32];
     // this thread's row of a P tile: keys half * 32 .. + 31 are 16-byte chunks
     // 4 half .. 4 half + 3 of a 128-byte row, stored at chunk c ^ (h & 7)
     const uint32_t p_row = smem_u32(smem + T::OFF_P) + (h >> 3) * 1024 + (h & 7) * 128;
-    for (int i = 0; i < n_blocks; ++i) {
-      // ---- logits of this warp's 32 keys; the S buffer is released at once.
-      // A failed wait does not leave the loop before the partner exchange:
-      // the two warps of a quarter meet at a named barrier every block and
-      // leave together when either has failed.
-      const int idx = idx_next;
-      idx_next = load_idx(i + 1);
-      const uint32_t vmask = __ballot_sync(0xffffffffu, idx >= 0 && idx < p.n_kv);
-      if (ok) ok = mbar_wait(s_full, i & 1);
-      tc_fence_after();
-      tmem_ld32(tmem_base + lane_addr + T::COL_S + half * 32, sr);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
-      // ---- block max over the 64 keys, shared with the partner warp
+    uint32_t g = 0;
+    bool ok = true;
+    bool q_loaded = false;       // Q of the current unit is already in place
+    for (int64_t u = u0; u < n_units && ok; u += du) {
+      const VhUnit w = vh_unit(p, u);
+      if (w.n_blocks == 0) {
+        write_empty(w);
+        continue;
+      }
+      if (!q_loaded) load_q(w);
+      q_loaded = false;
+      prefetch_unit(u + du);
+      float m_used = -INFINITY;   // running max (log2 domain) the P values are relative to
+      float l = 0.f;              // this warp's share of the sum of the fp32 p (LSE)
+      float l_mma = 0.f;          // ... of the bf16-rounded p the PV MMA used (normalises O)
+      auto load_idx = [&](int blk) -> int {
+        const int slot = w.slot_begin + blk * NK + half * 32 + lane;
+        return (blk < w.n_blocks && slot < w.slot_end) ? w.row_idx[slot] : -1;
+      };
+      int idx_next = load_idx(0);
+      for (int i = 0; i < w.n_blocks; ++i, ++g) {
+        // ---- logits of this warp's 32 keys; the S buffer is released at
+        // once. A failed wait does not leave the loop before the partner
+        // exchange: the two warps of a quarter meet at a named barrier every
+        // block and leave together when either has failed.
+        const int idx = idx_next;
+        idx_next = load_idx(i + 1);
+        const uint32_t vmask = __ballot_sync(0xffffffffu, idx >= 0 && idx < p.n_kv);
+        if (ok) ok = mbar_wait(s_full, g & 1);
+        tc_fence_after();
+        tmem_ld32(tmem_base + lane_addr + T::COL_S + half * 32, sr);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        // ---- block max over the 64 keys, shared with the partner warp
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        z[j] = ((vmask >> j) & 1u) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
-      float mx[4];
+        for (int j = 0; j < 32; ++j)
+          z[j] = ((vmask >> j) & 1u) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
+        float mx[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
-        mx[r] = fmaxf(fmaxf(fmaxf(z[r], z[r + 4]), fmaxf(z[r + 8], z[r + 12])),
-                      fmaxf(fmaxf(z[r + 16], z[r + 20]), fmaxf(z[r + 24], z[r + 28])));
-      const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      float* red_i = red + (i & 1) * (2 * T::M);
-      red_i[half * T::M + h] = hmax;
-      if (!named_bar_and(1u + static_cast<uint32_t>(quarter), 64u, ok)) {
+        for (int r = 0; r < 4; ++r)
+          mx[r] = fmaxf(fmaxf(fmaxf(z[r], z[r + 4]), fmaxf(z[r + 8], z[r + 12])),
+                        fmaxf(fmaxf(z[r + 16], z[r + 20]), fmaxf(z[r + 24], z[r + 28])));
+        const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        float* red_i = red + (g & 1) * (2 * T::M);
+        red_i[half * T::M + h] = hmax;
+        if (!named_bar_and(pair_bar, 64u, ok)) {
+          ok = false;
+          break;
+        }
+        const float bmax = fmaxf(hmax, red_i[(half ^ 1) * T::M + h]);
+        // ---- online softmax. Rescaling O needs PV(g - 1) finished; writing
+        // P buffer g & 1 needs PV(g - 2) finished (implied by PV(g - 1): the
+        // PV MMAs complete in issue order).
+        const bool grow = bmax > m_used + 8.0f;
+        const float m_new = grow ? bmax : m_used;
+        if (i > 0 && __any_sync(0xffffffffu, grow)) {
+          if (ok) ok = mbar_wait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1);
+          tc_fence_after();
+          const float alpha = grow ? ex2_approx(m_used - m_new) : 1.0f;
+#pragma unroll 1
+          for (int c = half * (T::VH / 2); c < (half + 1) * (T::VH / 2) && ok; c += 16) {
+            uint32_t o[16];
+            tmem_ld16(tmem_base + lane_addr + T::COL_O + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            tmem_st16(tmem_base + lane_addr + T::COL_O + c, o);
+          }
+          tmem_wait_st();
+          l *= alpha;
+          l_mma *= alpha;
+        } else if (g > 1 && ok) {
+          ok = mbar_wait(&pv_done[g & 1], ((g >> 1) & 1) ^ 1);
+        }
+        m_used = m_new;
+        uint32_t pk[16];
+        float ls[4] = {0.f, 0.f, 0.f, 0.f}, lm[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float p0 = ex2_approx(z[2 * j] - m_used);
+          const float p1 = ex2_approx(z[2 * j + 1] - m_used);
+          const __nv_bfloat162 pb2 = __floats2bfloat162_rn(p0, p1);
+          ls[j & 3] += p0 + p1;
+          lm[j & 3] += __low2float(pb2) + __high2float(pb2);
+          pk[j] = *reinterpret_cast<const uint32_t*>(&pb2);
+        }
+        float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        float lsum_mma = (lm[0] + lm[1]) + (lm[2] + lm[3]);
+        if (m_used == -INFINITY) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) pk[j] = 0u;
+          lsum = 0.f;
+          lsum_mma = 0.f;
+        }
+        l += lsum;
+        l_mma += lsum_mma;
+        const uint32_t pb = p_row + (g & 1) * T::P_BYTES;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          sts_v4(pb + (((4 * half + c) ^ (h & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                 pk[4 * c + 3]);
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[g & 1]);
+      }
+      // all softmax warps go on, or stop, together
+      if (!named_bar_and(kAllBar, kAllThreads, ok)) {
         ok = false;
         break;
       }
-      const float bmax = fmaxf(hmax, red_i[(half ^ 1) * T::M + h]);
-      // ---- online softmax. Rescaling O needs PV(i - 1) finished; writing
-      // P buffer i & 1 needs PV(i - 2) finished (implied by PV(i - 1): the
-      // PV MMAs complete in issue order).
-      const bool grow = bmax > m_used + 8.0f;
-      const float m_new = grow ? bmax : m_used;
-      if (i > 0 && __any_sync(0xffffffffu, grow)) {
-        ok = mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1);
-        tc_fence_after();
-        const float alpha = grow ? ex2_approx(m_used - m_new) : 1.0f;
+      // ---- the next unit's Q: this unit's S MMAs have all completed (the
+      // last S was loaded above), so its logits may start during this
+      // epilogue
+      for (int64_t un = u + du; un < n_units; un += du) {
+        const VhUnit wn = vh_unit(p, un);
+        if (wn.n_blocks == 0) continue;
+        load_q(wn);
+        q_loaded = true;
+        break;
+      }
+      // ---- epilogue: O of this unit, once its last PV has finished
+      ok = mbar_wait(&pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1);
+      tc_fence_after();
+      // The quarter's two warps add their halves of l and l_mma in the
+      // exchange buffer (the barrier above ended both warps' reads of their
+      // last block maxima; the one below precedes the next unit's first
+      // write).
+      red[half * T::M + h] = l;
+      red[(2 + half) * T::M + h] = l_mma;
+      named_bar_sync(pair_bar, 64u);
+      const float l_o = red[(half ^ 1) * T::M + h];
+      const float lm_o = red[(2 + (half ^ 1)) * T::M + h];
+      const bool pv_ok = ok;
+      named_bar_sync(pair_bar, 64u);
+      const float l_all = half == 0 ? l + l_o : l_o + l;
+      const float lm_all = half == 0 ? l_mma + lm_o : lm_o + l_mma;
+      // O / sum(rounded p) is an exact convex combination of the V rows with
+      // weights perturbed by the bf16 rounding of p (a component shared by
+      // the rows cancels); the LSE keeps the unrounded sum.
+      const bool has = pv_ok && l_all > 0.f && lm_all > 0.f;
+      const float inv_l = has ? 1.0f / lm_all : 0.f;
+      const uint32_t keep = has ? 0xffffffffu : 0u;   // masks undefined TMEM when empty
+      const float lse_v = has ? (m_used + log2f(l_all)) * 0.69314718055994531f : -INFINITY;
+      // O leaves through the P area (free: the last PV has finished) in
+      // 32 KB rounds of CW columns: each thread puts CW / 2 of its lane's
+      // scaled columns there (16-byte chunk c of row h at chunk c ^ (h & 7)),
+      // then the 256 threads store whole 16-byte chunks, a warp two rows of
+      // CW columns at a time.
+      const bool direct = p.splits == 1;
+      const bool bf16_out = direct && p.out_bf16;
+      const int esz = bf16_out ? 2 : 4;
+      const int CW = T::P_BYTES * 2 / (T::M * esz);        // 128 (bf16) or 64 (fp32) columns
+      const int row_bytes = CW * esz;                      // 256
+      uint8_t* obase;
+      if (direct) {
+        const size_t o_off = static_cast<size_t>(w.row) * p.H * T::DV + w.vh * T::VH;
+        obase = bf16_out ? reinterpret_cast<uint8_t*>(static_cast<__nv_bfloat16*>(p.out) + o_off)
+                         : reinterpret_cast<uint8_t*>(static_cast<float*>(p.out) + o_off);
+      } else {
+        const size_t part = static_cast<size_t>(w.row) * p.splits + w.split;
+        obase = reinterpret_cast<uint8_t*>(p.part_o + part * p.H * T::DV + w.vh * T::VH);
+      }
+      const size_t o_stride = static_cast<size_t>(T::DV) * esz;   // bytes between head rows
+      const uint32_t stage = smem_u32(smem + T::OFF_P);
 #pragma unroll 1
-        for (int c = half * (T::VH / 2); c < (half + 1) * (T::VH / 2) && ok; c += 16) {
+      for (int c0 = 0; c0 < T::VH; c0 += CW) {
+        const uint32_t srow = stage + h * row_bytes;
+#pragma unroll 1
+        for (int c = c0 + half * (CW / 2); c < c0 + (half + 1) * (CW / 2); c += 16) {
           uint32_t o[16];
           tmem_ld16(tmem_base + lane_addr + T::COL_O + c, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tmem_st16(tmem_base + lane_addr + T::COL_O + c, o);
-        }
-        tmem_wait_st();
-        l *= alpha;
-        l_mma *= alpha;
-      } else if (i > 1) {
-        ok = mbar_wait(&pv_done[i & 1], ((i >> 1) & 1) ^ 1);
-      }
-      m_used = m_new;
-      uint32_t pk[16];
-      float ls[4] = {0.f, 0.f, 0.f, 0.f}, lm[4] = {0.f, 0.f, 0.f, 0.f};
+          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j] & keep) * inv_l);
+          const int cc = (c - c0) * esz / 16;              // first 16-byte chunk in the row
+          if (bf16_out) {
+            uint32_t pkd[8];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float p0 = ex2_approx(z[2 * j] - m_used);
-        const float p1 = ex2_approx(z[2 * j + 1] - m_used);
-        const __nv_bfloat162 pb2 = __floats2bfloat162_rn(p0, p1);
-        ls[j & 3] += p0 + p1;
-        lm[j & 3] += __low2float(pb2) + __high2float(pb2);
-        pk[j] = *reinterpret_cast<const uint32_t*>(&pb2);
-      }
-      float lsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      float lsum_mma = (lm[0] + lm[1]) + (lm[2] + lm[3]);
-      if (m_used == -INFINITY) {
+            for (int j = 0; j < 8; ++j) {
+              const __nv_bfloat162 v =
+                  __floats2bfloat162_rn(__uint_as_float(o[2 * j]), __uint_as_float(o[2 * j + 1]));
+              pkd[j] = *reinterpret_cast<const uint32_t*>(&v);
+            }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) pk[j] = 0u;
-        lsum = 0.f;
-        lsum_mma = 0.f;
-      }
-      l += lsum;
-      l_mma += lsum_mma;
-      const uint32_t pb = p_row + (i & 1) * T::P_BYTES;
+            for (int q2 = 0; q2 < 2; ++q2)
+              sts_v4(srow + (((cc + q2) ^ (h & 7)) << 4), pkd[4 * q2], pkd[4 * q2 + 1],
+                     pkd[4 * q2 + 2], pkd[4 * q2 + 3]);
+          } else {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        sts_v4(pb + (((4 * half + c) ^ (h & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
-               pk[4 * c + 3]);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[i & 1]);
-    }
-    if (ok && n_blocks > 0) {
-      ok = mbar_wait(&pv_done[(n_blocks - 1) & 1], ((n_blocks - 1) >> 1) & 1);
-      tc_fence_after();
-    }
-    // Both warps of a quarter add their halves of l and l_mma (through the
-    // stage area: every gather and MMA has finished by now).
-    float* red_l = reinterpret_cast<float*>(smem + T::OFF_END);   // [half][2][128]
-    red_l[(half * 2) * T::M + h] = l;
-    red_l[(half * 2 + 1) * T::M + h] = l_mma;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&end_bar[quarter]);
-    ok = mbar_wait(&end_bar[quarter], 0) && ok;
-    const float l_o = red_l[((half ^ 1) * 2) * T::M + h];
-    const float lm_o = red_l[((half ^ 1) * 2 + 1) * T::M + h];
-    const float l_all = half == 0 ? l + l_o : l_o + l;
-    const float lm_all = half == 0 ? l_mma + lm_o : lm_o + l_mma;
-    // O / sum(rounded p) is an exact convex combination of the V rows with
-    // weights perturbed by the bf16 rounding of p (a component shared by the
-    // rows cancels); the LSE keeps the unrounded sum.
-    const bool has = ok && l_all > 0.f && lm_all > 0.f;
-    const float inv_l = has ? 1.0f / lm_all : 0.f;
-    const uint32_t keep = has ? 0xffffffffu : 0u;   // masks undefined TMEM when empty
-    const float lse_v = has ? (m_used + log2f(l_all)) * 0.69314718055994531f : -INFINITY;
-    // O leaves through the stage area (free now): each thread writes its
-    // row's 128 scaled columns there (16-byte chunk c of row h at chunk
-    // c ^ (h & 7)), then the eight softmax warps store whole rows, so every
-    // global store of a warp covers 512 contiguous bytes.
-    const bool direct = p.splits == 1;
-    const bool bf16_out = direct && p.out_bf16;
-    const int row_bytes = T::VH * (bf16_out ? 2 : 4);
-    const int n_chunks = row_bytes / 16;
-    uint8_t* o_stage = smem + T::OFF_OSTAGE;
-    {
-      const uint32_t row_base = smem_u32(o_stage) + h * row_bytes;
-#pragma unroll 1
-      for (int c = half * (T::VH / 2); c < (half + 1) * (T::VH / 2); c += 16) {
-        uint32_t o[16];
-        tmem_ld16(tmem_base + lane_addr + T::COL_O + c, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j] & keep) * inv_l);
-        if (bf16_out) {
-          uint32_t pkd[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const __nv_bfloat162 v =
-                __floats2bfloat162_rn(__uint_as_float(o[2 * j]), __uint_as_float(o[2 * j + 1]));
-            pkd[j] = *reinterpret_cast<const uint32_t*>(&v);
+            for (int q2 = 0; q2 < 4; ++q2)
+              sts_v4(srow + (((cc + q2) ^ (h & 7)) << 4), o[4 * q2], o[4 * q2 + 1], o[4 * q2 + 2],
+                     o[4 * q2 + 3]);
           }
-          const int c0 = c / 8;                  // 16-byte chunk of column c (bf16)
-#pragma unroll
-          for (int q = 0; q < 2; ++q)
-            sts_v4(row_base + (((c0 + q) ^ (h & 7)) << 4), pkd[4 * q], pkd[4 * q + 1],
-                   pkd[4 * q + 2], pkd[4 * q + 3]);
+        }
+        named_bar_sync(kAllBar, kAllThreads);
+        const int nch = row_bytes / 16;                    // 16 chunks per staged row
+#pragma unroll 4
+        for (int k = stid; k < p.H * nch; k += kAllThreads) {
+          const int r = k / nch, ch = k - r * nch;
+          const uint4 v = lds_v4(stage + r * row_bytes + ((ch ^ (r & 7)) << 4));
+          *reinterpret_cast<uint4*>(obase + r * o_stride + static_cast<size_t>(c0) * esz + ch * 16) = v;
+        }
+        named_bar_sync(kAllBar, kAllThreads);              // before the area is written again
+      }
+      if (w.vh == 0 && half == 0 && h < p.H) {
+        if (direct) {
+          if (p.lse) p.lse[static_cast<size_t>(w.row) * p.H + h] = lse_v;
         } else {
-          const int c0 = c / 4;                  // 16-byte chunk of column c (fp32)
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            sts_v4(row_base + (((c0 + q) ^ (h & 7)) << 4), o[4 * q], o[4 * q + 1], o[4 * q + 2],
-                   o[4 * q + 3]);
+          p.part_lse[(static_cast<size_t>(w.row) * p.splits + w.split) * p.H + h] = lse_v;
         }
       }
-    }
-    named_bar_sync(5u, 32u * T::SOFTMAX_WARPS);
-    {
-      uint8_t* dst_base;
-      size_t dst_row_stride;                     // bytes between head rows
-      if (direct) {
-        const size_t o_off = (static_cast<size_t>(row) * p.H) * T::DV + vh * T::VH;
-        dst_base = bf16_out ? reinterpret_cast<uint8_t*>(static_cast<__nv_bfloat16*>(p.out) + o_off)
-                            : reinterpret_cast<uint8_t*>(static_cast<float*>(p.out) + o_off);
-      } else {
-        const size_t part = static_cast<size_t>(row) * p.splits + split;
-        dst_base = reinterpret_cast<uint8_t*>(p.part_o + (part * p.H) * T::DV + vh * T::VH);
-      }
-      dst_row_stride = static_cast<size_t>(T::DV) * (bf16_out ? 2 : 4);
-      const int tid = threadIdx.x - 5 * 32;      // 0..255 over the softmax warps
-      const int total = p.H * n_chunks;
-#pragma unroll 4
-      for (int k = tid; k < total; k += 32 * T::SOFTMAX_WARPS) {
-        const int r = k / n_chunks, ch = k - r * n_chunks;
-        const uint4 v = lds_v4(smem_u32(o_stage) + r * row_bytes + ((ch ^ (r & 7)) << 4));
-        *reinterpret_cast<uint4*>(dst_base + r * dst_row_stride + ch * 16) = v;
-      }
-    }
-    if (vh == 0 && half == 0 && h < p.H) {
-      if (direct) {
-        if (p.lse) p.lse[static_cast<size_t>(row) * p.H + h] = lse_v;
-      } else {
-        p.part_lse[(static_cast<size_t>(row) * p.splits + split) * p.H + h] = lse_v;
-      }
+      // the TMEM loads of O are complete (wait::ld above) before this unit's
+      // successor writes its first P, which is what lets PV overwrite O; the
+      // eight warps agree on going on
+      ok = named_bar_and(kAllBar, kAllThreads, ok);
     }
   }
 
