@@ -582,15 +582,17 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
       const uint32_t keep = has ? 0xffffffffu : 0u;   // masks undefined TMEM when empty
       const float lse_v = has ? (m_used + log2f(l_all)) * 0.69314718055994531f : -INFINITY;
       // O leaves through the P area (free: the last PV has finished) in
-      // 32 KB rounds of CW columns: each thread puts CW / 2 of its lane's
-      // scaled columns there (16-byte chunk c of row h at chunk c ^ (h & 7)),
-      // then the 256 threads store whole 16-byte chunks, a warp two rows of
-      // CW columns at a time.
+      // rounds of CW columns, alternating between its two 16 KB halves: each
+      // thread puts CW / 2 of its lane's scaled columns there (16-byte chunk
+      // c of row h at chunk c ^ (h & 7)), then the 256 threads store whole
+      // 16-byte chunks, a warp four rows of CW columns at a time. One barrier
+      // per round: a half is written again only after the next round's
+      // barrier, which every thread reaches after its stores from that half.
       const bool direct = p.splits == 1;
       const bool bf16_out = direct && p.out_bf16;
       const int esz = bf16_out ? 2 : 4;
-      const int CW = T::P_BYTES * 2 / (T::M * esz);        // 128 (bf16) or 64 (fp32) columns
-      const int row_bytes = CW * esz;                      // 256
+      const int CW = T::P_BYTES / (T::M * esz);            // 64 (bf16) or 32 (fp32) columns
+      const int row_bytes = CW * esz;                      // 128
       uint8_t* obase;
       if (direct) {
         const size_t o_off = static_cast<size_t>(w.row) * p.H * T::DV + w.vh * T::VH;
@@ -601,10 +603,11 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
         obase = reinterpret_cast<uint8_t*>(p.part_o + part * p.H * T::DV + w.vh * T::VH);
       }
       const size_t o_stride = static_cast<size_t>(T::DV) * esz;   // bytes between head rows
-      const uint32_t stage = smem_u32(smem + T::OFF_P);
 #pragma unroll 1
-      for (int c0 = 0; c0 < T::VH; c0 += CW) {
+      for (int c0 = 0, rnd = 0; c0 < T::VH; c0 += CW, ++rnd) {
+        const uint32_t stage = smem_u32(smem + T::OFF_P) + (rnd & 1) * T::P_BYTES;
         const uint32_t srow = stage + h * row_bytes;
+        // this thread's CW / 2 columns, 16 at a time
 #pragma unroll 1
         for (int c = c0 + half * (CW / 2); c < c0 + (half + 1) * (CW / 2); c += 16) {
           uint32_t o[16];
@@ -612,7 +615,7 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j] & keep) * inv_l);
-          const int cc = (c - c0) * esz / 16;              // first 16-byte chunk in the row
+          const int cc = (c - c0) * esz / 16;              // its first 16-byte chunk in the row
           if (bf16_out) {
             uint32_t pkd[8];
 #pragma unroll
@@ -633,15 +636,18 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
           }
         }
         named_bar_sync(kAllBar, kAllThreads);
-        const int nch = row_bytes / 16;                    // 16 chunks per staged row
-#pragma unroll 4
-        for (int k = stid; k < p.H * nch; k += kAllThreads) {
-          const int r = k / nch, ch = k - r * nch;
-          const uint4 v = lds_v4(stage + r * row_bytes + ((ch ^ (r & 7)) << 4));
-          *reinterpret_cast<uint4*>(obase + r * o_stride + static_cast<size_t>(c0) * esz + ch * 16) = v;
+        constexpr int nch = 8;                             // 16-byte chunks per staged row
+#pragma unroll
+        for (int m = 0; m < T::M * nch / kAllThreads; ++m) {
+          const int k = stid + m * kAllThreads;
+          const int r = k >> 3, ch = k & 7;
+          if (r < p.H) {
+            const uint4 v = lds_v4(stage + r * row_bytes + ((ch ^ (r & 7)) << 4));
+            *reinterpret_cast<uint4*>(obase + r * o_stride + static_cast<size_t>(c0) * esz + ch * 16) = v;
+          }
         }
-        named_bar_sync(kAllBar, kAllThreads);              // before the area is written again
       }
+      named_bar_sync(kAllBar, kAllThreads);                // the P area is free again
       if (w.vh == 0 && half == 0 && h < p.H) {
         if (direct) {
           if (p.lse) p.lse[static_cast<size_t>(w.row) * p.H + h] = lse_v;
