@@ -370,12 +370,32 @@ dsa_status launch_indexer_topk(const dsa_shape* s, const HostLayout& lay, const 
   return DSA_OK;
 }
 
+// A launch that may overlap the previous kernel of the stream (programmatic
+// stream serialization); the kernel waits (griddep_wait) before it reads
+// anything that kernel writes. Used only for the second and later kernels of
+// dsa_forward, whose first kernel is an ordinary launch.
+template <class... Params, class... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, int smem,
+                             cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ------------------------------------------------------------------ top-k launch
 
 dsa_status launch_topk(const dsa_shape* s, const HostLayout& lay, const float* scores,
                        int32_t row_begin, int32_t rows, const int32_t* q_pos0,
                        const int32_t* kv_len, int32_t* indices, int32_t out_rows,
-                       int32_t out_row0, cudaStream_t stream, int dev) {
+                       int32_t out_row0, cudaStream_t stream, int dev, bool dependent = false) {
   static std::atomic<bool> attr_done[kMaxDevices];
   const int smem = static_cast<int>(sizeof(dsa::TopkSmem));
   if (dsa_status st = set_smem(dsa::topk_kernel, smem, dev, attr_done)) return st;
@@ -392,7 +412,11 @@ dsa_status launch_topk(const dsa_shape* s, const HostLayout& lay, const float* s
   p.out_rows = out_rows;
   p.out_row0 = out_row0;
   dim3 grid(2 * rows, s->batch);   // a cluster of two CTAs per row
-  dsa::topk_kernel<<<grid, dsa::kTopkThreads, smem, stream>>>(p);
+  if (dependent)
+    DSA_CUDA_TRY(launch_dependent(dsa::topk_kernel, grid, dim3(dsa::kTopkThreads), smem, stream, p),
+                 "top-k launch");
+  else
+    dsa::topk_kernel<<<grid, dsa::kTopkThreads, smem, stream>>>(p);
   DSA_CUDA_TRY(cudaGetLastError(), "top-k launch");
   return DSA_OK;
 }
@@ -478,7 +502,7 @@ dsa_status launch_attn_t(const dsa_shape* s, const dsa::KeyMap& km, const AttnPl
 dsa_status launch_attn_vh(const dsa_shape* s, const dsa::KeyMap& km, const AttnPlan& pl,
                           const uint16_t* q, const uint16_t* kv, const int32_t* indices,
                           void* out, int out_bf16, float* lse, void* ws, cudaStream_t stream,
-                          int dev) {
+                          int dev, bool dependent) {
   using T = dsa::VhTile;
   static std::atomic<bool> attr_done[kMaxDevices];
   if (dsa_status st = set_smem(dsa::sparse_attn_vh_kernel, T::SMEM_BYTES, dev, attr_done))
@@ -510,8 +534,13 @@ dsa_status launch_attn_vh(const dsa_shape* s, const dsa::KeyMap& km, const AttnP
   const int64_t n_units = rows * pl.splits * 2;
   if (n_units >= (1ll << 31)) return fail(DSA_ERR_INVALID_ARG, "too many attention rows");
   const int64_t grid = std::min<int64_t>(n_units, std::max(2, num_sms() / 2 * 2));
-  dsa::sparse_attn_vh_kernel<<<static_cast<unsigned>(grid), T::THREADS, T::SMEM_BYTES, stream>>>(
-      p, n_units);
+  if (dependent)
+    DSA_CUDA_TRY(launch_dependent(dsa::sparse_attn_vh_kernel, dim3(static_cast<unsigned>(grid)),
+                                  dim3(T::THREADS), T::SMEM_BYTES, stream, p, n_units),
+                 "sparse attention launch");
+  else
+    dsa::sparse_attn_vh_kernel<<<static_cast<unsigned>(grid), T::THREADS, T::SMEM_BYTES, stream>>>(
+        p, n_units);
   DSA_CUDA_TRY(cudaGetLastError(), "sparse attention launch");
   if (pl.splits > 1) {
     dim3 grid(static_cast<unsigned>(rows), s->heads);
@@ -523,7 +552,8 @@ dsa_status launch_attn_vh(const dsa_shape* s, const dsa::KeyMap& km, const AttnP
 
 dsa_status launch_attn(const dsa_shape* s, const dsa::KeyMap& km, const uint16_t* q,
                        const uint16_t* kv, const int32_t* indices, void* out, int out_bf16,
-                       float* lse, void* ws, size_t ws_bytes, cudaStream_t stream, int dev) {
+                       float* lse, void* ws, size_t ws_bytes, cudaStream_t stream, int dev,
+                       bool dependent = false) {
   const AttnPlan pl = plan_attn(s);
   if (pl.ws_bytes > 0) {
     if (!ws || ws_bytes < pl.ws_bytes)
@@ -532,7 +562,8 @@ dsa_status launch_attn(const dsa_shape* s, const dsa::KeyMap& km, const uint16_t
     if (!aligned(ws, 256)) return fail(DSA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
   }
   if (s->qk_dim == 576)
-    return launch_attn_vh(s, km, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
+    return launch_attn_vh(s, km, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev,
+                          dependent);
   return launch_attn_t<64, 64, 1>(s, km, pl, q, kv, indices, out, out_bf16, lse, ws, stream, dev);
 }
 
@@ -985,13 +1016,17 @@ dsa_status dsa_forward_ex(const dsa_shape* s, const dsa_layout* layout, const ui
     if (dsa_status e = launch_indexer(s, lay, q_fp8, q_scale, w, k_fp8, k_scale, q_pos0, kv_len,
                                       r0, rows, scores, 0, st_, dev))
       return e;
-    // The chunk's selections go straight to their rows of indices_out.
+    // The chunk's selections go straight to their rows of indices_out. The
+    // top-k and the attention are dependent launches: each may start its
+    // set-up while the kernel before it finishes, and waits for that kernel
+    // before reading its output; the indexer is an ordinary launch (the
+    // scores buffer it writes is read by the previous chunk's top-k).
     if (dsa_status e = launch_topk(s, lay, scores, r0, rows, q_pos0, kv_len, indices_out, s->n_q,
-                                   r0, st_, dev))
+                                   r0, st_, dev, true))
       return e;
   }
   return launch_attn(s, lay.km, q, kv, indices_out, out, out_dtype == DSA_OUT_BF16, lse, attn_ws,
-                     f.attn_bytes, st_, dev);
+                     f.attn_bytes, st_, dev, true);
 }
 
 dsa_status dsa_forward(const dsa_shape* s, const uint8_t* q_fp8, const float* q_scale,

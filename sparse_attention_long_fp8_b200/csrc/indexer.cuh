@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(IndexerTile<HI, DI, QG>::THREADS, 1)
                     static_cast<int32_t>(y >= 0 ? y : p.km.pool_rows));
         ++issued;
       }
+      griddep_launch_dependents();   // the top-k may start its set-up
       // Drain: every issued key tile has landed before the CTA may exit.
       for (int i = max(0, issued - T::STAGES); i < issued; ++i)
         mbar_wait(&k_full[i % T::STAGES], (i / T::STAGES) & 1);

@@ -199,6 +199,7 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
     using BV = std::integral_constant<bool, true>;
     uint32_t g = 0;
     bool ok = true;
+    griddep_wait();               // the indices may come from the previous kernel
     for (int64_t u = u0; u < n_units && ok; u += du) {
       const VhUnit w = vh_unit(p, u);
       auto load_keys = [&](int blk, int64_t (&k)[4]) {
@@ -409,6 +410,7 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
     };
     // A unit without blocks (a split past the top-k slots): O = 0, LSE = -inf.
     auto write_empty = [&](const VhUnit& w) {
+      griddep_wait();
       if (h >= p.H) return;
       const bool direct = p.splits == 1;
       for (int c = half * (T::VH / 2); c < (half + 1) * (T::VH / 2); ++c) {
@@ -444,7 +446,10 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
         write_empty(w);
         continue;
       }
-      if (!q_loaded) load_q(w);
+      if (!q_loaded) {
+        load_q(w);
+        griddep_wait();           // the indices may come from the previous kernel
+      }
       q_loaded = false;
       prefetch_unit(u + du);
       float m_used = -INFINITY;   // running max (log2 domain) the P values are relative to

@@ -133,6 +133,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTopkThreads, 1)
   extern __shared__ __align__(16) uint8_t tk_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_raw);
 
+  // the scores come from the previous kernel (launched with a dependent
+  // launch in the forward path)
+  griddep_wait();
   const int r = blockIdx.x >> 1, b = blockIdx.y;
   const uint32_t part = cluster_ctarank();     // which half of the row this CTA scans
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -144,6 +147,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTopkThreads, 1)
   const uint32_t k = static_cast<uint32_t>(p.k);
 
   if (n <= p.k) {   // both CTAs of the pair leave here (same row, same n)
+    griddep_launch_dependents();
     if (part == 0)
       for (int i = tid; i < p.k; i += kTopkThreads) out[i] = i < n ? i : -1;
     return;
@@ -243,6 +247,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTopkThreads, 1)
   }
   // ---- CTA 0 takes CTA 1's candidates behind its own
   cluster_sync();                  // both candidate buffers and counts are final
+  griddep_launch_dependents();     // the attention may start its own set-up
   if (part != 0) {
     cluster_sync();                // CTA 0 has read this CTA's shared memory
     return;
