@@ -475,16 +475,24 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(s_free);
-        // ---- block max over the 64 keys, shared with the partner warp
+        // ---- block max over the 64 keys, shared with the partner warp. The
+        // logits stay unscaled in z: the scale is positive, so the maximum
+        // of the scaled logits is the scaled maximum (rounding is monotone),
+        // and p = 2^(z * scale - m) is one fma. Keys outside the set (a warp-
+        // uniform test, rare) are -inf.
 #pragma unroll
-        for (int j = 0; j < 32; ++j)
-          z[j] = ((vmask >> j) & 1u) ? __uint_as_float(sr[j]) * p.scale_log2 : -INFINITY;
+        for (int j = 0; j < 32; ++j) z[j] = __uint_as_float(sr[j]);
+        if (vmask != 0xffffffffu) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (!((vmask >> j) & 1u)) z[j] = -INFINITY;
+        }
         float mx[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r)
           mx[r] = fmaxf(fmaxf(fmaxf(z[r], z[r + 4]), fmaxf(z[r + 8], z[r + 12])),
                         fmaxf(fmaxf(z[r + 16], z[r + 20]), fmaxf(z[r + 24], z[r + 28])));
-        const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        const float hmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
         float* red_i = red + (g & 1) * (2 * T::M);
         red_i[half * T::M + h] = hmax;
         if (!named_bar_and(pair_bar, 64u, ok)) {
@@ -521,8 +529,8 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
         float ls[4] = {0.f, 0.f, 0.f, 0.f}, lm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float p0 = ex2_approx(z[2 * j] - m_used);
-          const float p1 = ex2_approx(z[2 * j + 1] - m_used);
+          const float p0 = ex2_approx(fmaf(z[2 * j], p.scale_log2, -m_used));
+          const float p1 = ex2_approx(fmaf(z[2 * j + 1], p.scale_log2, -m_used));
           const __nv_bfloat162 pb2 = __floats2bfloat162_rn(p0, p1);
           ls[j & 3] += p0 + p1;
           lm[j & 3] += __low2float(pb2) + __high2float(pb2);
