@@ -595,7 +595,8 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
       const uint32_t keep = has ? 0xffffffffu : 0u;   // masks undefined TMEM when empty
       const float lse_v = has ? (m_used + log2f(l_all)) * 0.69314718055994531f : -INFINITY;
       // O leaves through the P area (free: the last PV has finished) in
-      // rounds of CW columns, alternating between its two 16 KB halves: each
+      // rounds of CW columns, alternating between its two 16 KB halves (or,
+      // after the CTA's last unit, through the stage area at once): each
       // thread puts CW / 2 of its lane's scaled columns there (16-byte chunk
       // c of row h at chunk c ^ (h & 7)), then the 256 threads store whole
       // 16-byte chunks, a warp four rows of CW columns at a time. One barrier
@@ -604,8 +605,12 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
       const bool direct = p.splits == 1;
       const bool bf16_out = direct && p.out_bf16;
       const int esz = bf16_out ? 2 : 4;
-      const int CW = T::P_BYTES / (T::M * esz);            // 64 (bf16) or 32 (fp32) columns
-      const int row_bytes = CW * esz;                      // 128
+      // After the CTA's last unit nothing is gathered any more: the stage
+      // area takes all of O in one round.
+      const bool last = !q_loaded;
+      const int CW = last ? T::VH : T::P_BYTES / (T::M * esz);   // columns per round
+      const int row_bytes = CW * esz;
+      const int nch_log2 = __ffs(row_bytes / 16) - 1;      // 16-byte chunks per staged row
       uint8_t* obase;
       if (direct) {
         const size_t o_off = static_cast<size_t>(w.row) * p.H * T::DV + w.vh * T::VH;
@@ -618,7 +623,8 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
       const size_t o_stride = static_cast<size_t>(T::DV) * esz;   // bytes between head rows
 #pragma unroll 1
       for (int c0 = 0, rnd = 0; c0 < T::VH; c0 += CW, ++rnd) {
-        const uint32_t stage = smem_u32(smem + T::OFF_P) + (rnd & 1) * T::P_BYTES;
+        const uint32_t stage =
+            last ? smem_u32(c_smem) : smem_u32(smem + T::OFF_P) + (rnd & 1) * T::P_BYTES;
         const uint32_t srow = stage + h * row_bytes;
         // this thread's CW / 2 columns, 16 at a time
 #pragma unroll 1
@@ -649,11 +655,9 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
           }
         }
         named_bar_sync(kAllBar, kAllThreads);
-        constexpr int nch = 8;                             // 16-byte chunks per staged row
-#pragma unroll
-        for (int m = 0; m < T::M * nch / kAllThreads; ++m) {
-          const int k = stid + m * kAllThreads;
-          const int r = k >> 3, ch = k & 7;
+#pragma unroll 4
+        for (int k = stid; k < (T::M << nch_log2); k += kAllThreads) {
+          const int r = k >> nch_log2, ch = k & ((1 << nch_log2) - 1);
           if (r < p.H) {
             const uint4 v = lds_v4(stage + r * row_bytes + ((ch ^ (r & 7)) << 4));
             *reinterpret_cast<uint4*>(obase + r * o_stride + static_cast<size_t>(c0) * esz + ch * 16) = v;
