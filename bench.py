@@ -399,8 +399,8 @@ def breakdown(step, steps):
 # q read once plus out and lse written once (the latent gathers hit L2), so it
 # grows in proportion to the rows and is scaled by them. When the source no
 # longer matches, the figure is stale and the line reports null.
-ATTN_TRAFFIC_4K = {"bytes": 642.317568e6 + 1022.450e6, "rows": 4096,
-                   "source_sha256": "c3490702679e4156ad68ead2d99bb67c2fe9078e35829ef9665883c60fd2d25d"}
+ATTN_TRAFFIC_4K = {"bytes": 642.480128e6 + 1023.750e6, "rows": 4096,
+                   "source_sha256": "e606947ea9f5cc0682b8a0d653266ea0800e4c57506b13738fb3cd0d5d063b4d"}
 
 
 def kernel_source_sha256(name):
