@@ -134,6 +134,23 @@ dsa_status make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint3
   return DSA_OK;
 }
 
+// 2D byte tensor [rows, row_bytes] with a box of [box_rows, 128 bytes] and
+// the 128-byte swizzle (the attention's output stores).
+dsa_status make_tmap_rows128(CUtensorMap* map, void* base, uint64_t rows, uint32_t row_bytes,
+                             uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[2] = {row_bytes, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return DSA_OK;
+}
+
 // ------------------------------------------------------------------ validation
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -529,6 +546,17 @@ dsa_status launch_attn_vh(const dsa_shape* s, const dsa::KeyMap& km, const AttnP
     p.part_o = static_cast<float*>(ws);
     p.part_lse = reinterpret_cast<float*>(static_cast<char*>(ws) + (po + 255) / 256 * 256);
   }
+  // the output as rows of DV elements for the kernel's TMA stores
+  CUtensorMap to;
+  {
+    const bool direct = pl.splits == 1;
+    const uint32_t esz = (direct && out_bf16) ? 2u : 4u;
+    const uint64_t orows = static_cast<uint64_t>(rows) * (direct ? 1 : pl.splits) * s->heads;
+    if (dsa_status st = make_tmap_rows128(&to, direct ? out : static_cast<void*>(p.part_o), orows,
+                                          static_cast<uint32_t>(s->v_dim) * esz,
+                                          static_cast<uint32_t>(s->heads)))
+      return st;
+  }
   // persistent CTAs (one per SM, an even number so that a CTA keeps its
   // value half), each walking units c, c + grid, ...
   const int64_t n_units = rows * pl.splits * 2;
@@ -536,11 +564,11 @@ dsa_status launch_attn_vh(const dsa_shape* s, const dsa::KeyMap& km, const AttnP
   const int64_t grid = std::min<int64_t>(n_units, std::max(2, num_sms() / 2 * 2));
   if (dependent)
     DSA_CUDA_TRY(launch_dependent(dsa::sparse_attn_vh_kernel, dim3(static_cast<unsigned>(grid)),
-                                  dim3(T::THREADS), T::SMEM_BYTES, stream, p, n_units),
+                                  dim3(T::THREADS), T::SMEM_BYTES, stream, to, p, n_units),
                  "sparse attention launch");
   else
     dsa::sparse_attn_vh_kernel<<<static_cast<unsigned>(grid), T::THREADS, T::SMEM_BYTES, stream>>>(
-        p, n_units);
+        to, p, n_units);
   DSA_CUDA_TRY(cudaGetLastError(), "sparse attention launch");
   if (pl.splits > 1) {
     dim3 grid(static_cast<unsigned>(rows), s->heads);

@@ -114,7 +114,11 @@ __device__ __forceinline__ VhUnit vh_unit(const AttnParams& p, int64_t u) {
 // the logit MMAs and owns TMEM; 5-12 run the softmax (two warps per TMEM lane
 // quarter: a thread owns one head row and 32 of a block's 64 keys); 13 issues
 // the PV MMAs.
-__global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, int64_t n_units) {
+// tmap_o: the output (p.out, or p.part_o in split mode) as a byte tensor of
+// rows of DV elements, one row per (row, head) (or (row, split, head)), box
+// 128 bytes x H rows with the 128-byte swizzle.
+__global__ void __launch_bounds__(448, 1)
+    sparse_attn_vh_kernel(const __grid_constant__ CUtensorMap tmap_o, AttnParams p, int64_t n_units) {
   using T = VhTile;
   constexpr int NK = T::NK;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -594,77 +598,73 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
       const float inv_l = has ? 1.0f / lm_all : 0.f;
       const uint32_t keep = has ? 0xffffffffu : 0u;   // masks undefined TMEM when empty
       const float lse_v = has ? (m_used + log2f(l_all)) * 0.69314718055994531f : -INFINITY;
-      // O leaves through the P area (free: the last PV has finished) in
-      // rounds of CW columns, alternating between its two 16 KB halves (or,
-      // after the CTA's last unit, through the stage area at once): each
-      // thread puts CW / 2 of its lane's scaled columns there (16-byte chunk
-      // c of row h at chunk c ^ (h & 7)), then the 256 threads store whole
-      // 16-byte chunks, a warp four rows of CW columns at a time. One barrier
-      // per round: a half is written again only after the next round's
-      // barrier, which every thread reaches after its stores from that half.
+      // O leaves by TMA stores of 128-byte-wide column slices (32 fp32 or 64
+      // bf16 columns, 16 KB for 128 rows) staged in the swizzled layout the
+      // store reads (16-byte chunk c of row h at h * 128 + ((c ^ (h & 7)) <<
+      // 4)); each thread stages half of a slice's columns of its row. One
+      // slice per round, alternating between the two P buffers (free: the
+      // last PV has finished); after the CTA's last unit (nothing is
+      // gathered any more) all slices at once through the stage area. The
+      // stores run on while the warps go on; a buffer is written again only
+      // after the store that read it has finished reading.
       const bool direct = p.splits == 1;
       const bool bf16_out = direct && p.out_bf16;
       const int esz = bf16_out ? 2 : 4;
-      // After the CTA's last unit nothing is gathered any more: the stage
-      // area takes all of O in one round.
+      const int slice_cols = 128 / esz;
+      const int n_slices = T::VH / slice_cols;
       const bool last = !q_loaded;
-      const int CW = last ? T::VH : T::P_BYTES / (T::M * esz);   // columns per round
-      const int row_bytes = CW * esz;
-      const int nch_log2 = __ffs(row_bytes / 16) - 1;      // 16-byte chunks per staged row
-      uint8_t* obase;
-      if (direct) {
-        const size_t o_off = static_cast<size_t>(w.row) * p.H * T::DV + w.vh * T::VH;
-        obase = bf16_out ? reinterpret_cast<uint8_t*>(static_cast<__nv_bfloat16*>(p.out) + o_off)
-                         : reinterpret_cast<uint8_t*>(static_cast<float*>(p.out) + o_off);
-      } else {
-        const size_t part = static_cast<size_t>(w.row) * p.splits + w.split;
-        obase = reinterpret_cast<uint8_t*>(p.part_o + part * p.H * T::DV + w.vh * T::VH);
-      }
-      const size_t o_stride = static_cast<size_t>(T::DV) * esz;   // bytes between head rows
+      const int per_round = last ? n_slices : 1;
+      const int32_t y_row = static_cast<int32_t>(
+          (direct ? static_cast<int64_t>(w.row) : static_cast<int64_t>(w.row) * p.splits + w.split) *
+          p.H);
 #pragma unroll 1
-      for (int c0 = 0, rnd = 0; c0 < T::VH; c0 += CW, ++rnd) {
+      for (int s0 = 0, rnd = 0; s0 < n_slices; s0 += per_round, ++rnd) {
         const uint32_t stage =
             last ? smem_u32(c_smem) : smem_u32(smem + T::OFF_P) + (rnd & 1) * T::P_BYTES;
-        const uint32_t srow = stage + h * row_bytes;
-        // this thread's CW / 2 columns, 16 at a time
+        if (!last && stid == 0) bulk_wait_read<1>();     // the store of round rnd - 2 has read it
+        named_bar_sync(kAllBar, kAllThreads);
+        for (int sl = s0; sl < s0 + per_round; ++sl) {
+          const uint32_t srow = stage + (sl - s0) * (T::M * 128) + h * 128;
 #pragma unroll 1
-        for (int c = c0 + half * (CW / 2); c < c0 + (half + 1) * (CW / 2); c += 16) {
-          uint32_t o[16];
-          tmem_ld16(tmem_base + lane_addr + T::COL_O + c, o);
-          tmem_wait_ld();
+          for (int c = half * (slice_cols / 2); c < (half + 1) * (slice_cols / 2); c += 16) {
+            uint32_t o[16];
+            tmem_ld16(tmem_base + lane_addr + T::COL_O + sl * slice_cols + c, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j] & keep) * inv_l);
-          const int cc = (c - c0) * esz / 16;              // its first 16-byte chunk in the row
-          if (bf16_out) {
-            uint32_t pkd[8];
+            for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j] & keep) * inv_l);
+            const int cc = c * esz / 16;                   // its first 16-byte chunk in the row
+            if (bf16_out) {
+              uint32_t pkd[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const __nv_bfloat162 v =
-                  __floats2bfloat162_rn(__uint_as_float(o[2 * j]), __uint_as_float(o[2 * j + 1]));
-              pkd[j] = *reinterpret_cast<const uint32_t*>(&v);
+              for (int j = 0; j < 8; ++j) {
+                const __nv_bfloat162 v =
+                    __floats2bfloat162_rn(__uint_as_float(o[2 * j]), __uint_as_float(o[2 * j + 1]));
+                pkd[j] = *reinterpret_cast<const uint32_t*>(&v);
+              }
+#pragma unroll
+              for (int q2 = 0; q2 < 2; ++q2)
+                sts_v4(srow + (((cc + q2) ^ (h & 7)) << 4), pkd[4 * q2], pkd[4 * q2 + 1],
+                       pkd[4 * q2 + 2], pkd[4 * q2 + 3]);
+            } else {
+#pragma unroll
+              for (int q2 = 0; q2 < 4; ++q2)
+                sts_v4(srow + (((cc + q2) ^ (h & 7)) << 4), o[4 * q2], o[4 * q2 + 1], o[4 * q2 + 2],
+                       o[4 * q2 + 3]);
             }
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2)
-              sts_v4(srow + (((cc + q2) ^ (h & 7)) << 4), pkd[4 * q2], pkd[4 * q2 + 1],
-                     pkd[4 * q2 + 2], pkd[4 * q2 + 3]);
-          } else {
-#pragma unroll
-            for (int q2 = 0; q2 < 4; ++q2)
-              sts_v4(srow + (((cc + q2) ^ (h & 7)) << 4), o[4 * q2], o[4 * q2 + 1], o[4 * q2 + 2],
-                     o[4 * q2 + 3]);
           }
         }
+        fence_proxy_async_smem();
         named_bar_sync(kAllBar, kAllThreads);
-#pragma unroll 4
-        for (int k = stid; k < (T::M << nch_log2); k += kAllThreads) {
-          const int r = k >> nch_log2, ch = k & ((1 << nch_log2) - 1);
-          if (r < p.H) {
-            const uint4 v = lds_v4(stage + r * row_bytes + ((ch ^ (r & 7)) << 4));
-            *reinterpret_cast<uint4*>(obase + r * o_stride + static_cast<size_t>(c0) * esz + ch * 16) = v;
-          }
+        if (stid == 0) {
+          for (int sl = s0; sl < s0 + per_round; ++sl)
+            tma_store_2d(&tmap_o, stage + (sl - s0) * (T::M * 128),
+                         (w.vh * T::VH + sl * slice_cols) * esz, y_row);
+          bulk_commit();
         }
       }
-      named_bar_sync(kAllBar, kAllThreads);                // the P area is free again
+      // every staged byte read before the next unit writes P (or gathers)
+      if (stid == 0) bulk_wait_read<0>();
+      named_bar_sync(kAllBar, kAllThreads);
       if (w.vh == 0 && half == 0 && h < p.H) {
         if (direct) {
           if (p.lse) p.lse[static_cast<size_t>(w.row) * p.H + h] = lse_v;
@@ -679,6 +679,7 @@ __global__ void __launch_bounds__(448, 1) sparse_attn_vh_kernel(AttnParams p, in
     }
   }
 
+  if (threadIdx.x == 5 * 32) bulk_wait<0>();   // the output stores have completed
   tc_fence_before();
   __syncthreads();
   if (warp == 4) {
