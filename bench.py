@@ -399,8 +399,8 @@ def breakdown(step, steps):
 # q read once plus out and lse written once (the latent gathers hit L2), so it
 # grows in proportion to the rows and is scaled by them. When the source no
 # longer matches, the figure is stale and the line reports null.
-ATTN_TRAFFIC_4K = {"bytes": 642.480128e6 + 1023.750e6, "rows": 4096,
-                   "source_sha256": "e606947ea9f5cc0682b8a0d653266ea0800e4c57506b13738fb3cd0d5d063b4d"}
+ATTN_TRAFFIC_4K = {"bytes": 642.971648e6 + 1023.432e6, "rows": 4096,
+                   "source_sha256": "f4bf1014203b94cb30eae110a2f2f972f5711f62954f3b00d92e2e247ea55dab"}
 
 
 def kernel_source_sha256(name):
