@@ -26,7 +26,12 @@
  *     device's primary context): the cached state would be stale.
  *   - Every call is asynchronous on the caller's CUDA stream (`stream`, a
  *     cudaStream_t passed as void*; NULL = legacy default stream). No call
- *     synchronises except dsa_check().
+ *     synchronises except dsa_check(). Inside dsa_forward[_ex], the top-k
+ *     and attention kernels that follow a score kernel are programmatic
+ *     dependent launches (they may start their set-up while the kernel
+ *     before them finishes, and wait for it before reading its output); the
+ *     first kernel of every call is an ordinary launch, so every call is
+ *     ordered after the caller's earlier work on the stream as usual.
  *   - Argument errors are detected on the host BEFORE any launch and reported
  *     by the return value; dsa_last_error() gives a one-line reason.
  *   - Device-side failures (a bounded wait that ran out) set a per-device
