@@ -109,10 +109,12 @@ def _random_scores(rows, n_kv, seed, ties=True):
 
 @pytest.mark.parametrize("n_kv,k,pos0", [(300, 64, 0), (300, 64, 200), (4096, 2048, 4090),
                                            (5000, 2048, 2044), (50000, 2048, 49994),
-                                           (70000, 100, 69994)])
+                                           (70000, 100, 69994), (40001, 2048, 39995)])
 def test_topk_exact_on_given_scores(n_kv, k, pos0):
     """Integer work: on the same fp32 scores the selection must equal the
-    oracle's (ties to the lower index) exactly."""
+    oracle's (ties to the lower index) exactly. With an odd n_kv every row
+    but the first starts off a 16-byte boundary and takes the scalar scan;
+    the all-equal row overflows the candidate buffers (the fallback)."""
     rows = 6
     cfg = dsa_inputs.custom_config("prefill_4k", n_q=pos0 + rows, n_kv=n_kv, topk=k, name="tk")
     s32 = _random_scores(rows, n_kv, seed=n_kv)
