@@ -399,8 +399,8 @@ def breakdown(step, steps):
 # q read once plus out and lse written once (the latent gathers hit L2), so it
 # grows in proportion to the rows and is scaled by them. When the source no
 # longer matches, the figure is stale and the line reports null.
-ATTN_TRAFFIC_4K = {"bytes": 642.971648e6 + 1023.432e6, "rows": 4096,
-                   "source_sha256": "f4bf1014203b94cb30eae110a2f2f972f5711f62954f3b00d92e2e247ea55dab"}
+ATTN_TRAFFIC_4K = {"bytes": 642.458624e6 + 1022.275e6, "rows": 4096,
+                   "source_sha256": "576884927b8853594d6ee7f667b2a6e341b0b8ebaa4b53573f4b85f8bb4a35f6"}
 
 
 def kernel_source_sha256(name):

@@ -35,8 +35,7 @@
 // The CTAs are persistent: CTA c takes units c, c + grid, ... (a unit is one
 // (query row, split, value half)), and every barrier phase runs on across
 // units. At the end of a unit the softmax warps load the next unit's Q (its
-// S MMAs can then start) before they write this unit's O, and the next
-// unit's Q row is prefetched into L2 while the current unit runs.
+// S MMAs can then start) before they write this unit's O.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -403,15 +402,6 @@ __global__ void __launch_bounds__(448, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(q_ready);
     };
-    // The next unit's Q rows into L2 (a hint): 256 threads, one line each
-    // per step.
-    auto prefetch_unit = [&](int64_t u) {
-      if (u >= n_units) return;
-      const VhUnit w = vh_unit(p, u);
-      const char* q = reinterpret_cast<const char*>(p.q + static_cast<size_t>(w.row) * p.H * T::DQK);
-      const int lines = p.H * T::DQK * 2 / 128;
-      for (int l = stid; l < lines; l += kAllThreads) prefetch_l2(q + static_cast<size_t>(l) * 128);
-    };
     // A unit without blocks (a split past the top-k slots): O = 0, LSE = -inf.
     auto write_empty = [&](const VhUnit& w) {
       griddep_wait();
@@ -455,7 +445,6 @@ __global__ void __launch_bounds__(448, 1)
         griddep_wait();           // the indices may come from the previous kernel
       }
       q_loaded = false;
-      prefetch_unit(u + du);
       float m_used = -INFINITY;   // running max (log2 domain) the P values are relative to
       float l = 0.f;              // this warp's share of the sum of the fp32 p (LSE)
       float l_mma = 0.f;          // ... of the bf16-rounded p the PV MMA used (normalises O)
